@@ -1,0 +1,618 @@
+#!/usr/bin/env python
+"""Benchmark of the paged-KV-cache attention hot path on B200.
+
+One step = one pass of the hot path over one batch of synthetic inputs that
+already sit in HBM.  The default workload is the Llama-2-7B-shaped MHA decode
+step: the cache append of the 64 new K/V rows (random slot mapping) followed
+by decode attention of 64 sequences (32/32 heads, head_dim 128, bf16, page
+16, contexts uniform in [512, 4096]), split-KV partitions and their merge
+included.  ``--workload`` selects the other workloads (GQA decode, long
+context bf16/INT8, chunked prefill with a shared prefix, tiny fp32 decode).
+
+Prints ONE JSON line (rank 0).  ``value`` is whole-job throughput: algorithmic
+bytes (decode) or flops (prefill) of all ranks' steps divided by the device
+time of the timed steps (CUDA events on the launching stream, max over ranks).
+``e2e`` repeats the measurement through the public API from pinned host
+buffers, with the per-step host->device copies of the step's inputs and the
+device->host copy of its output inside the timed region.  ``roofline`` is for
+the dominant kernel (the decode or prefill call), timed with CUDA events
+around that call inside the timed steps.  ``cpu_baseline`` times the fp64
+oracle on the host cores (rank 0, N = 1 only).
+
+``--impl reference`` times the fp64 CPU oracle (the reference arm here) on a
+bounded sample of the same workload and prints the same line shape.
+
+Multi-GPU (torchrun): each rank runs an independent replica of the workload
+(the decode and prefill paths shard over sequences with no exchange step), so
+scaling is weak and there is no data-path collective; ranks only meet at the
+barriers around the timed region and in the max/sum of the timings.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention HBM GB/s (% of 8 TB/s), tokens/s; prefill TFLOP/s"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic per launch of the dominant kernel from an ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), keyed by workload, with the
+# hash of the kernel sources it was taken on; reported only while they match.
+TRAFFIC = {}
+KERNEL_SOURCES = {
+    "decode": ["paged_kv_cache_380_b200/csrc/decode.cu", "paged_kv_cache_380_b200/csrc/pkv_ptx.cuh",
+               "paged_kv_cache_380_b200/csrc/pkv_common.cuh"],
+    "prefill": ["paged_kv_cache_380_b200/csrc/prefill.cu", "paged_kv_cache_380_b200/csrc/pkv_ptx.cuh",
+                "paged_kv_cache_380_b200/csrc/pkv_common.cuh"],
+}
+
+
+def kernel_sha(kind: str) -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES[kind]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---- distributed plumbing (host logic; tested on CPU with gloo) ------------------
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def aggregate(elapsed_ms: float, units: float, work: float, group=None):
+    """Max of the timed region over ranks and sums of units/work over ranks."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return elapsed_ms, units, work
+    dev = "cuda" if dist.get_backend(group) == "nccl" else "cpu"
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    s = torch.tensor([units, work], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    dist.all_reduce(s, op=dist.ReduceOp.SUM, group=group)
+    return float(t.item()), float(s[0].item()), float(s[1].item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# ---- clock sampling during the timed region (NVML reads only) ---------------------
+
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+           0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+           0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Polls the SM clock and clock-event reasons of this process's GPU every
+    few milliseconds in a background thread (read-only NVML queries)."""
+
+    def __init__(self, torch_device: int, period_s: float = 0.005):
+        self.samples = []
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        self.max_mhz = None
+        self.handle = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(torch_device)
+            bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+            self._nvml = pynvml
+        except Exception as e:  # pragma: no cover - reported, not fatal
+            self.error = repr(e)
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                try:
+                    reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                except AttributeError:
+                    reasons = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.handle)
+                self.samples.append((time.perf_counter(), mhz, reasons))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.handle is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+            time.sleep(0.05)
+
+    def stop(self):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self, t0: float, t1: float):
+        if self.handle is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "error", "")}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not inside and self.samples:        # very short region: nearest samples around it
+            inside = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:3]
+        mask = 0
+        for s in inside:
+            mask |= s[2]
+        names = [n for bit, n in REASONS.items() if mask & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(s[1] for s in inside) if inside else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(inside)}
+
+
+# ---- workloads -----------------------------------------------------------------------
+
+def dev(a, tag):
+    import numpy as np
+    import torch
+    a = np.ascontiguousarray(a)
+    if tag == "bf16":
+        return torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+    if tag == "f16":
+        return torch.from_numpy(a.view(np.float16)).cuda()
+    return torch.from_numpy(a).cuda()
+
+
+class DecodeStep:
+    """Cache append of the new rows (when the workload has them) + decode."""
+
+    kind = "decode"
+
+    def __init__(self, case, int8: bool = False):
+        import numpy as np
+        import torch
+        from paged_kv_cache_380_b200 import ops
+        self.case, self.int8 = case, int8
+        tag = case.dtype
+        B, Hq, D = case.q.shape
+        P, ps, Hkv, _ = case.k_pages.shape
+        self.q = dev(case.q, tag)
+        self.bt = dev(case.block_tables, "i32")
+        self.cl = dev(case.context_lens, "i32")
+        self.out = torch.empty_like(self.q)
+        if int8:
+            kb, vb = dev(case.k_pages, tag), dev(case.v_pages, tag)
+            self.kp = torch.empty(kb.shape, dtype=torch.int8, device="cuda")
+            self.vp = torch.empty_like(self.kp)
+            self.ks = torch.empty(kb.shape[:3], dtype=torch.float16, device="cuda")
+            self.vs = torch.empty_like(self.ks)
+            ident = torch.arange(P * ps, dtype=torch.int64, device="cuda")
+            ops.kv_cache_write_quant(kb.view(P * ps, Hkv, D), vb.view(P * ps, Hkv, D), ident, self.kp, self.vp,
+                                     self.ks, self.vs)
+            del kb, vb
+            torch.cuda.synchronize()
+            elem, scale_bytes = 1, 2
+        else:
+            self.kp, self.vp = dev(case.k_pages, tag), dev(case.v_pages, tag)
+            self.ks = self.vs = None
+            elem, scale_bytes = (4 if tag == "f32" else 2), 0
+        self.has_new = case.k_new is not None and not int8
+        if self.has_new:
+            self.k_new, self.v_new = dev(case.k_new, tag), dev(case.v_new, tag)
+            self.slots = dev(case.slot_mapping, "i64")
+        kvdt = torch.int8 if int8 else self.kp.dtype
+        self.splits, self.split_tokens = ops.decode_plan(B, Hq, Hkv, D, ps, case.max_pages_per_seq, kvdt)
+        need = ops.decode_workspace_size(B, Hq, Hkv, D, ps, case.max_pages_per_seq, kvdt)
+        self.ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
+        qelem = 4 if tag == "f32" else 2
+        ctx = case.context_lens.astype(np.int64)
+        pages = int(np.sum((ctx + ps - 1) // ps))
+        # algorithmic bytes: every cached K/V element read once (+ its scale for INT8),
+        # q read, out written, block-table entries and context lengths read
+        self.decode_bytes = (int(ctx.sum()) * Hkv * (2 * D * elem + 2 * scale_bytes)
+                             + 2 * B * Hq * D * qelem + pages * 4 + B * 4)
+        self.write_bytes = 0
+        if self.has_new:
+            T = case.k_new.shape[0]
+            self.write_bytes = 2 * 2 * T * Hkv * D * elem + T * 8
+        self.work = self.decode_bytes + self.write_bytes       # bytes per step
+        self.units = B                                          # sequences advanced one token
+        self.launches = (1 if self.has_new else 0) + 1 + (1 if self.splits > 1 else 0)
+        self.in_l2 = self.work > 4 * L2_BYTES
+
+    def run(self, ev=None):
+        from paged_kv_cache_380_b200 import ops
+        if self.has_new:
+            ops.kv_cache_write(self.k_new, self.v_new, self.slots, self.kp, self.vp)
+        if ev is not None:
+            ev[0].record()
+        ops.paged_attention_decode(self.q, self.kp, self.vp, self.bt, self.cl, self.case.scale, self.out,
+                                   k_scales=self.ks, v_scales=self.vs, workspace=self.ws)
+        if ev is not None:
+            ev[1].record()
+
+    def host_io(self):
+        """Pinned host copies of the per-step inputs and the output buffer."""
+        import torch
+        ins = [self.q, self.bt, self.cl] + ([self.k_new, self.v_new, self.slots] if self.has_new else [])
+        hosts = [t.cpu().pin_memory() for t in ins]
+        out_h = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        return list(zip(hosts, ins)), out_h
+
+    def config(self):
+        c = self.case
+        B, Hq, D = c.q.shape
+        return {"workload": c.name + ("_int8" if self.int8 else ""), "batch": B, "num_q_heads": Hq,
+                "num_kv_heads": c.num_kv_heads, "head_dim": D, "page_size": c.page_size,
+                "kv_dtype": "i8" if self.int8 else c.dtype, "mean_context": float(c.context_lens.mean()),
+                "num_pages": c.num_pages, "splits": self.splits, "split_tokens": self.split_tokens,
+                "new_tokens_written": int(c.k_new.shape[0]) if self.has_new else 0,
+                "l2": ("inputs larger than L2 (%.2f GB read per step vs 126 MB L2)" % (self.work / 1e9))}
+
+
+class PrefillStep:
+    """Cache append of the chunk's K/V, then causal chunked prefill."""
+
+    kind = "prefill"
+
+    def __init__(self, case):
+        import numpy as np
+        import torch
+        self.case = case
+        tag = case.dtype
+        self.q = dev(case.q, tag)
+        self.kp, self.vp = dev(case.k_pages, tag), dev(case.v_pages, tag)
+        self.bt, self.qs, self.cl = dev(case.block_tables, "i32"), dev(case.q_start, "i32"), dev(case.context_lens, "i32")
+        self.k_new, self.v_new, self.slots = dev(case.k_new, tag), dev(case.v_new, tag), dev(case.slot_mapping, "i64")
+        self.out = torch.empty_like(self.q)
+        self.max_q = int(np.max(np.diff(case.q_start)))
+        Hq, D = case.num_q_heads, case.head_dim
+        n = np.diff(case.q_start).astype(np.int64)
+        ctx = case.context_lens.astype(np.int64)
+        # keys attended per (row, head): ctx - n + r + 1 for r < n
+        keys = int(np.sum(n * (ctx - n) + n * (n + 1) // 2))
+        self.work = 4.0 * D * Hq * keys           # flops per step (QK^T and PV, 2 flops per MAC)
+        self.units = int(n.sum())                  # query rows processed
+        self.launches = 2
+        self.flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+
+    def before_step(self):
+        self.flush.fill_(1)                        # L2 flush (outside the per-step events)
+
+    def run(self, ev=None):
+        from paged_kv_cache_380_b200 import ops
+        ops.kv_cache_write(self.k_new, self.v_new, self.slots, self.kp, self.vp)
+        if ev is not None:
+            ev[0].record()
+        ops.paged_attention_prefill(self.q, self.kp, self.vp, self.bt, self.qs, self.cl, True, self.case.scale,
+                                    self.out, max_q_len=self.max_q)
+        if ev is not None:
+            ev[1].record()
+
+    def host_io(self):
+        import torch
+        ins = [self.q, self.bt, self.qs, self.cl, self.k_new, self.v_new, self.slots]
+        hosts = [t.cpu().pin_memory() for t in ins]
+        out_h = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        return list(zip(hosts, ins)), out_h
+
+    def config(self):
+        c = self.case
+        return {"workload": c.name, "num_seqs": c.batch, "chunk": int(np.diff(c.q_start)[0]) if c.batch else 0,
+                "context": int(c.context_lens[0]), "shared_prefix_pages": c.meta.get("shared_pages"),
+                "num_q_heads": c.num_q_heads, "num_kv_heads": c.num_kv_heads, "head_dim": c.head_dim,
+                "page_size": c.page_size, "l2": "L2 flushed between steps (252 MB write outside the events)"}
+
+
+def make_step(name: str):
+    from paged_kv_cache_380_b200 import workloads as W
+    if name == "long_ctx_split_kv_int8":
+        return DecodeStep(W.long_ctx_split_kv(), int8=True)
+    case = W.WORKLOADS[name]()
+    return PrefillStep(case) if case.kind == "prefill" else DecodeStep(case)
+
+
+# ---- the GPU arm ------------------------------------------------------------------------
+
+def time_steps(step, K, events=True):
+    """Run K steps, per-step CUDA events; returns (total_ms, dominant_ms_list)."""
+    import torch
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    dom = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for i in range(K):
+        if hasattr(step, "before_step"):
+            step.before_step()
+        starts[i].record()
+        step.run(dom[i] if events else None)
+        ends[i].record()
+    torch.cuda.synchronize()
+    total = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    dom_ms = [a.elapsed_time(b) for a, b in dom] if events else []
+    return total, dom_ms
+
+
+def time_e2e(step, K):
+    import torch
+    pairs, out_h = step.host_io()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    h2d = sum(h.numel() * h.element_size() for h, _ in pairs)
+    d2h = out_h.numel() * out_h.element_size()
+    for i in range(K):
+        if hasattr(step, "before_step"):
+            step.before_step()
+        starts[i].record()
+        for h, d in pairs:
+            d.copy_(h, non_blocking=True)
+        step.run()
+        out_h.copy_(step.out, non_blocking=True)
+        ends[i].record()
+    torch.cuda.synchronize()
+    return sum(s.elapsed_time(e) for s, e in zip(starts, ends)), h2d, d2h
+
+
+def cpu_baseline(step, budget_s: float = 20.0):
+    """The fp64 oracle on the host cores over a bounded sample of the workload."""
+    import oracle
+    c = step.case
+    threads = oracle.max_threads()
+    if step.kind == "decode":
+        B = c.batch
+        # sample: the first S sequences (all heads), S sized to ~budget from a 1-sequence probe
+        t0 = time.perf_counter()
+        items = np.arange(c.num_q_heads)
+        _run_oracle_decode(step, items)
+        one = max(time.perf_counter() - t0, 1e-3)
+        S = int(max(1, min(B, budget_s / one / 2)))
+        items = np.arange(S * c.num_q_heads)
+        t0 = time.perf_counter()
+        _run_oracle_decode(step, items)
+        dt = time.perf_counter() - t0
+        frac = c.context_lens[:S].astype(np.int64).sum() / c.context_lens.astype(np.int64).sum()
+        work = step.decode_bytes * frac
+        return {"value": work / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                "sample": f"decode of the first {S} of {B} sequences, all {c.num_q_heads} heads, fp64 "
+                          f"({dt:.1f} s)", "seconds": dt}
+    T = c.q.shape[0]
+    Hq = c.num_q_heads
+    rng = np.random.default_rng(0)
+    t0 = time.perf_counter()
+    probe = rng.choice(T * Hq, 64, replace=False)
+    _run_oracle_prefill(step, probe)
+    per = max((time.perf_counter() - t0) / 64, 1e-6)
+    n = int(min(T * Hq, max(64, budget_s / per / 2)))
+    items = rng.choice(T * Hq, n, replace=False)
+    t0 = time.perf_counter()
+    _run_oracle_prefill(step, items)
+    dt = time.perf_counter() - t0
+    work = step.work * n / (T * Hq)
+    return {"value": work / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"prefill of {n} random (row, head) items of {T * Hq}, fp64 ({dt:.1f} s)", "seconds": dt}
+
+
+def _run_oracle_decode(step, items):
+    import oracle
+    c = step.case
+    if step.int8:
+        if not hasattr(step, "_q8"):
+            step._q8 = (*oracle.quantize_int8(c.k_pages, c.dtype), *oracle.quantize_int8(c.v_pages, c.dtype))
+        kq, ks, vq, vs = step._q8
+        return oracle.decode(c.q, c.dtype, kq, vq, "i8", c.block_tables, c.context_lens, c.scale,
+                             k_scales=ks, v_scales=vs, items=items)
+    k, v = c.k_pages, c.v_pages
+    if step.has_new:
+        k, v = k.copy(), v.copy()
+        oracle.kv_cache_write(c.k_new, c.v_new, c.slot_mapping, k, v)
+    return oracle.decode(c.q, c.dtype, k, v, c.dtype, c.block_tables, c.context_lens, c.scale, items=items)
+
+
+def _run_oracle_prefill(step, items):
+    import oracle
+    c = step.case
+    k, v = c.k_pages.copy(), c.v_pages.copy()
+    oracle.kv_cache_write(c.k_new, c.v_new, c.slot_mapping, k, v)
+    return oracle.prefill(c.q, c.dtype, k, v, c.dtype, c.block_tables, c.q_start, c.context_lens, True,
+                          c.scale, items=items)
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    from paged_kv_cache_380_b200 import ops
+    ops.load()
+    step = make_step(args.workload)
+    K, W = args.steps, max(3, args.warmup)
+    for _ in range(W):
+        if hasattr(step, "before_step"):
+            step.before_step()
+        step.run()
+    torch.cuda.synchronize()
+    code, detail = ops.device_status()
+    if code != 0:
+        raise RuntimeError(f"device status after warm-up: {ops.error_string(code)} ({detail})")
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.perf_counter()
+    total_ms, dom_ms = time_steps(step, K)
+    torch.cuda.synchronize()
+    t_wall1 = time.perf_counter()
+    barrier()
+    sampler.stop()
+    clocks = sampler.summary(t_wall0, t_wall1)
+
+    elapsed, units, work = aggregate(total_ms, step.units * K, step.work * K)
+
+    # end to end from pinned host buffers (same metric)
+    barrier()
+    torch.cuda.synchronize()
+    e2e_ms, h2d, d2h = time_e2e(step, K)
+    e2e_ms, _, _ = aggregate(e2e_ms, 0, 0)
+    barrier()
+    code, detail = ops.device_status()
+    if code != 0:
+        raise RuntimeError(f"device status after timing: {ops.error_string(code)} ({detail})")
+
+    peaks, peak_src = load_peaks()
+    scale_div = 1e9 if step.kind == "decode" else 1e12
+    unit = "GB/s" if step.kind == "decode" else "TFLOP/s"
+    value = work / (elapsed / 1e3) / scale_div
+    dom_avg_ms = statistics.mean(dom_ms)
+    if step.kind == "decode":
+        dom_work = step.decode_bytes
+        peak = peaks["hbm_gbs"]
+        achieved = dom_work / (dom_avg_ms / 1e3) / 1e9
+        bound, runit = "hbm", "GB/s"
+    else:
+        dom_work = step.work
+        peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        achieved = dom_work / (dom_avg_ms / 1e3) / 1e12
+        bound, runit = "tensor", "TFLOP/s"
+    tr = TRAFFIC.get(config_key(args.workload))
+    traffic = tr["bytes"] if tr and tr["kernel_sha"] == kernel_sha(step.kind) else None
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": round(elapsed / K, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "i8" if getattr(step, "int8", False) else step.case.dtype,
+        "data": "synthetic (seeded N(0,1) inputs, shuffled physical pages)",
+        "config": dict(step.config(), parallelism=f"replicas{world}" if world > 1 else "single-gpu"),
+        "impl": "ours",
+        "extra": ({"tokens_per_s": round(units / (elapsed / 1e3), 1),
+                   "pct_of_8TBps": round(100 * value / 8000.0, 2)} if step.kind == "decode"
+                  else {"rows_per_s": round(units / (elapsed / 1e3), 1)}),
+        "roofline": {"bound": bound, "achieved": round(achieved, 3), "peak": peak, "unit": runit,
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "kernel": ("decode call (main kernel + split-KV merge)" if step.kind == "decode"
+                                else "prefill kernel"),
+                     "kernel_ms": round(dom_avg_ms, 5), "peak_source": f"{peak_src} (MEASURED_PEAKS.json)"
+                     if peak_src == "measured" else "fallback"},
+        "e2e": {"value": round(work / (e2e_ms / 1e3) / scale_div, 3), "unit": unit,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / K, 5)},
+        "gpu_launches": step.launches * K,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(step, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def config_key(name):
+    return name
+
+
+def run_reference(args):
+    """The fp64 CPU oracle as the reference arm (rank 0 only)."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    from paged_kv_cache_380_b200 import workloads as W
+    name = args.workload
+    int8 = name == "long_ctx_split_kv_int8"
+    case = W.long_ctx_split_kv() if int8 else W.WORKLOADS[name]()
+
+    class HostStep:
+        pass
+    step = HostStep()
+    step.case, step.int8, step.kind = case, int8, case.kind
+    step.has_new = case.k_new is not None and not int8
+    K, Wm = args.steps, max(3, args.warmup)
+    if case.kind == "decode":
+        S = max(1, min(case.batch, args.ref_seqs))
+        items = np.arange(S * case.num_q_heads)
+        Hkv, D = case.num_kv_heads, case.head_dim
+        elem = 1 if int8 else (4 if case.dtype == "f32" else 2)
+        ctx = case.context_lens[:S].astype(np.int64)
+        work = int(ctx.sum()) * Hkv * (2 * D * elem + (4 if int8 else 0)) + 2 * S * case.num_q_heads * D * 2
+        fn = lambda: _run_oracle_decode(step, items)  # noqa: E731
+        div, unit, units = 1e9, "GB/s", S
+        sample = f"decode of the first {S} of {case.batch} sequences (all heads) per step"
+    else:
+        T, Hq = case.q.shape[0], case.num_q_heads
+        n = min(T * Hq, args.ref_items)
+        items = np.random.default_rng(0).choice(T * Hq, n, replace=False)
+        nn = np.diff(case.q_start).astype(np.int64)
+        ctx = case.context_lens.astype(np.int64)
+        keys = int(np.sum(nn * (ctx - nn) + nn * (nn + 1) // 2))
+        work = 4.0 * case.head_dim * Hq * keys * n / (T * Hq)
+        fn = lambda: _run_oracle_prefill(step, items)  # noqa: E731
+        div, unit, units = 1e12, "TFLOP/s", n
+        sample = f"prefill of {n} random (row, head) items per step"
+    for _ in range(Wm):
+        fn()
+    t0 = time.perf_counter()
+    for _ in range(K):
+        fn()
+    dt = time.perf_counter() - t0
+    value = work * K / dt / div
+    line = {"metric": METRIC, "value": round(value, 6), "unit": unit, "n_gpus": world, "steps": K, "warmup": Wm,
+            "ms_per_step": round(dt / K * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) inputs, shuffled physical pages)",
+            "config": {"workload": name, "parallelism": "host cores"}, "impl": "reference",
+            "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": oracle.max_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama2_7b_mha_decode",
+                    choices=["tiny_decode_f32", "llama2_7b_mha_decode", "llama2_70b_gqa_decode",
+                             "long_ctx_split_kv", "long_ctx_split_kv_int8", "chunked_prefill_shared_prefix"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0, help="CPU-baseline sample budget")
+    ap.add_argument("--ref-seqs", type=int, default=4, help="reference arm: sequences per step (decode)")
+    ap.add_argument("--ref-items", type=int, default=512, help="reference arm: (row, head) items per step")
+    args = ap.parse_args(argv)
+    rank, world, _ = dist_env()
+    if args.gpus != world and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,513 @@
+// Decode attention over a paged KV cache: one query token per sequence.
+//
+// What is computed: out[b][h] = softmax(scale * q[b][h] . K_b^T) V_b over all
+// context_lens[b] cached tokens ("大模型推理优化：KV Cache与FlashAttention实战"
+// §2.1; "大模型推理优化实战：KV Cache + Flash Attention，让 Token 生成快 3 倍",
+// "KV Cache 的工作原理"), K_b/V_b read page by page through the block table
+// ("Flash Attention与Paged KV Cache优化大模型计算效率" §3.2), query head h using
+// KV head h / G ("LLM推理系统优化：KV缓存管理与动态批处理技术" §2.1, GQA).  The
+// softmax is evaluated tile by tile with the online recurrence of the page
+// "KV Cache + Flash Attention，让 Token 生成快 3 倍" ("Flash Attention 的分块计算
+// 原理": running max m, running sum l, accumulator rescaled by exp(m_old -
+// m_new)); the division by l happens once at the end (the printed loop divides
+// inside the loop as well, which double-normalises; the plain reading is the
+// standard recurrence).  Softmax state and accumulators are fp32 ("大模型推理优化：
+// KV Cache与FlashAttention实战" §6), exponentials in base 2 with log2(e) folded
+// into the scale.
+//
+// B200 design (HBM-bound: every K/V byte is read once, ~1-8 flop per byte):
+//  * CTA = (partition, KV head, sequence); its WARPS warps take the
+//    partition's 16-token chunks round-robin, each warp with a private
+//    STAGES-deep cp.async ring (16-byte copies, zero-filled past the context)
+//    so ~100 KB per SM is in flight.  Page tiles land XOR-swizzled (16-byte
+//    unit u of row r at u ^ (r & 7)) so ldmatrix reads are bank-conflict free.
+//  * All G query heads of the KV head share each K/V tile.  Both contractions
+//    run on the tensor cores with the context as the M dimension, so no group
+//    size wastes rows:  S^T[16 tok x 8 heads] = K[16 x D] . Q^T and
+//    O^T[D x 8 heads] += V^T[D x 16 tok] . P^T; P^T's fragments come from S^T's
+//    accumulator by an 8x8 movmatrix transpose.  Max/sum across the chunk use
+//    warp shuffles.
+//  * INT8 pages (one fp16 scale per token and KV head, the symmetric
+//    quantisation of "LLM推理系统优化" §3.2): codes are widened exactly to the
+//    MMA type in registers; the key scale multiplies the score of its token,
+//    the value scale multiplies that token's probability before P.V.  The
+//    d-axis is permuted consistently in Q and K (and in V and the output) so
+//    that each thread's ldmatrix bytes form whole MMA fragments.
+//  * Long contexts are split into partitions of whole chunks (split-KV); each
+//    CTA writes its normalised partial and log-sum-exp, and a second kernel
+//    merges them: lse = log2 sum 2^lse_p, out = sum_p 2^(lse_p - lse) o_p.
+#include <cmath>
+#include <type_traits>
+
+#include "pkv_kernels.h"
+#include "pkv_ptx.cuh"
+
+namespace pkv {
+namespace {
+
+constexpr int kChunk = 16;            // tokens per pipeline stage of one warp
+constexpr unsigned kFull = 0xffffffffu;
+
+// int8 code pair (bytes a, b of w) -> two MMA-type values, exact: the byte,
+// offset by 128, becomes the low mantissa bits of 2^23 (fp32), then the offset
+// is subtracted; |code| <= 128 is exact in bf16 and fp16.
+template <typename QT>
+__device__ __forceinline__ uint32_t s8pair(uint32_t w_biased, uint32_t sel_a, uint32_t sel_b) {
+    const float fa = __int_as_float(__byte_perm(w_biased, 0x4B000000u, 0x7540u | sel_a)) - 8388736.0f;
+    const float fb = __int_as_float(__byte_perm(w_biased, 0x4B000000u, 0x7540u | sel_b)) - 8388736.0f;
+    return pack2<QT>(fa, fb);
+}
+
+template <typename QT>
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+    if constexpr (std::is_same<QT, __nv_bfloat16>::value)
+        ptx::mma_bf16_16816(d, a0, a1, a2, a3, b0, b1);
+    else
+        ptx::mma_f16_16816(d, a0, a1, a2, a3, b0, b1);
+}
+
+template <typename QT, typename KVT, int HD, int NT, int WARPS, int STAGES>
+struct DecodeCfg {
+    static constexpr bool kInt8 = std::is_same<KVT, int8_t>::value;
+    static constexpr int kRowBytes = HD * static_cast<int>(sizeof(KVT));
+    static constexpr int kUnits = kRowBytes / 16;
+    static constexpr int kTile = kChunk * kRowBytes;
+    static constexpr int kScaleBytes = kInt8 ? 2 * kChunk * 4 : 0;
+    static constexpr int kStage = 2 * kTile + kScaleBytes;
+    static constexpr int kPipe = WARPS * STAGES * kStage;
+    static constexpr int kMerge = WARPS * 8 * NT * (HD + 2) * 4;
+    static constexpr int kSmem = kPipe > kMerge ? kPipe : kMerge;
+    static constexpr int kDT = HD / 16;   // 16-wide d tiles (MMA k-steps for QK, M tiles for PV)
+    static_assert(kUnits >= 8, "rows must span at least 128 bytes for the swizzle");
+    static_assert(!kInt8 || HD == 128, "INT8 pages need head_dim 128");
+};
+
+template <typename QT, typename KVT, int HD, int NT, int WARPS, int STAGES>
+__global__ void __launch_bounds__(WARPS * 32)
+decode_mma_kernel(const DecodeParams p) {
+    using Cfg = DecodeCfg<QT, KVT, HD, NT, WARPS, STAGES>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, c = lane & 3;
+    const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+    const int Hq = p.num_q_heads, Hkv = p.num_kv_heads, G = Hq / Hkv, ps = p.page_size;
+
+    const int ctx = __ldg(p.context_lens + b);
+    if (ctx < 0 || ctx > p.max_pages_per_seq * ps) {
+        if (split == 0 && kvh == 0 && threadIdx.x == 0) record_error(p.status, PKV_ERR_DEVICE_RANGE, ctx);
+        return;
+    }
+    QT* out = static_cast<QT*>(p.out);
+    const size_t head0 = static_cast<size_t>(b) * Hq + static_cast<size_t>(kvh) * G;
+    if (ctx == 0) {
+        if (split == 0)
+            for (int i = threadIdx.x; i < G * HD; i += WARPS * 32) out[head0 * HD + i] = from_float<QT>(0.f);
+        return;
+    }
+    const int n_chunks = ceil_div(ctx, kChunk);
+    const int nsplit = ceil_div(n_chunks, p.chunks_per_split);
+    if (split >= nsplit) return;
+    const int c_begin = split * p.chunks_per_split;
+    const int c_end = min(c_begin + p.chunks_per_split, n_chunks);
+    const int n_mine = (c_end - c_begin > warp) ? ceil_div(c_end - c_begin - warp, WARPS) : 0;
+
+    // ---- query fragments (B operand of S^T = K . Q^T), kept in registers ----
+    uint32_t qf[NT][Cfg::kDT][2];
+    {
+        const QT* q = static_cast<const QT*>(p.q);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int n = nt * 8 + g;
+            const QT* qrow = q + (head0 + n) * HD;
+#pragma unroll
+            for (int kk = 0; kk < Cfg::kDT; ++kk) {
+                const int d0 = Cfg::kInt8 ? kk * 16 + 4 * c : kk * 16 + 2 * c;
+                const int d1 = Cfg::kInt8 ? d0 + 2 : d0 + 8;
+                qf[nt][kk][0] = n < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + d0)) : 0u;
+                qf[nt][kk][1] = n < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + d1)) : 0u;
+            }
+        }
+    }
+
+    // ---- per-warp cp.async ring ----
+    uint8_t* ring = smem + warp * STAGES * Cfg::kStage;
+    const uint32_t ring_s = ptx::smem_u32(ring);
+    const uint8_t* kpool = static_cast<const uint8_t*>(p.k_pages);
+    const uint8_t* vpool = static_cast<const uint8_t*>(p.v_pages);
+    const int32_t* bt = p.block_tables + static_cast<size_t>(b) * p.max_pages_per_seq;
+    int page_reg = 0;
+
+    auto issue = [&](int i) {
+        if (i < n_mine) {
+            if ((i & 31) == 0) {        // page indices of my next 32 chunks, one per lane
+                const int j = i + lane;
+                page_reg = j < n_mine ? __ldg(bt + ((c_begin + warp + j * WARPS) * kChunk) / ps) : 0;
+            }
+            const int page = __shfl_sync(kFull, page_reg, i & 31);
+            const int tok0 = (c_begin + warp + i * WARPS) * kChunk;
+            const bool page_ok = page >= 0 && page < p.num_pages;
+            if (!page_ok && lane == 0) record_error(p.status, PKV_ERR_DEVICE_RANGE, page);
+            const int64_t row0 = (static_cast<int64_t>(page) * ps + (tok0 % ps)) * Hkv + kvh;
+            const uint32_t sK = ring_s + (i % STAGES) * Cfg::kStage;
+            const uint32_t sV = sK + Cfg::kTile;
+#pragma unroll
+            for (int x = lane; x < kChunk * Cfg::kUnits; x += 32) {
+                const int r = x / Cfg::kUnits, u = x % Cfg::kUnits;
+                const bool ok = page_ok && (tok0 + r < ctx);
+                const int64_t off = (row0 + static_cast<int64_t>(r) * Hkv) * Cfg::kRowBytes + u * 16;
+                const uint32_t dst = r * Cfg::kRowBytes + ((u ^ (r & 7)) << 4);
+                ptx::cp_async16(sK + dst, ok ? kpool + off : kpool, ok ? 16u : 0u);
+                ptx::cp_async16(sV + dst, ok ? vpool + off : vpool, ok ? 16u : 0u);
+            }
+            if constexpr (Cfg::kInt8) {   // lanes 0-15: key scales, 16-31: value scales
+                const int r = lane & 15;
+                const bool ok = page_ok && (tok0 + r < ctx);
+                const __half* sc = lane < 16 ? p.k_scales : p.v_scales;
+                const uintptr_t a = reinterpret_cast<uintptr_t>(sc + (row0 + static_cast<int64_t>(r) * Hkv));
+                ptx::cp_async4(sV + Cfg::kTile + lane * 4,
+                               ok ? reinterpret_cast<const void*>(a & ~uintptr_t(3)) : static_cast<const void*>(sc),
+                               ok ? 4u : 0u);
+            }
+        }
+        ptx::cp_async_commit();
+    };
+
+    float m[NT][2], l[NT][2], o[NT][Cfg::kDT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        m[nt][0] = m[nt][1] = -INFINITY;
+        l[nt][0] = l[nt][1] = 0.f;
+#pragma unroll
+        for (int dt = 0; dt < Cfg::kDT; ++dt) o[nt][dt][0] = o[nt][dt][1] = o[nt][dt][2] = o[nt][dt][3] = 0.f;
+    }
+
+#pragma unroll
+    for (int i = 0; i < STAGES - 1; ++i) issue(i);
+
+    for (int i = 0; i < n_mine; ++i) {
+        issue(i + STAGES - 1);
+        ptx::cp_async_wait<STAGES - 1>();
+        __syncwarp();
+        const uint32_t sK = ring_s + (i % STAGES) * Cfg::kStage;
+        const uint32_t sV = sK + Cfg::kTile;
+        const int tok0 = (c_begin + warp + i * WARPS) * kChunk;
+
+        // ---- S^T = K . Q^T  (16 tokens x 8 heads per n-tile) ----
+        float s[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+        {
+            const int r = lane & 15;
+            if constexpr (!Cfg::kInt8) {
+#pragma unroll
+                for (int kk = 0; kk < Cfg::kDT; ++kk) {
+                    const int u = 2 * kk + (lane >> 4);
+                    uint32_t a0, a1, a2, a3;
+                    ptx::ldmatrix_x4(sK + r * Cfg::kRowBytes + ((u ^ (r & 7)) << 4), a0, a1, a2, a3);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma16816<QT>(s[nt], a0, a1, a2, a3, qf[nt][kk][0], qf[nt][kk][1]);
+                }
+            } else {
+#pragma unroll
+                for (int U = 0; U < Cfg::kUnits; U += 2) {
+                    const int u = U + (lane >> 4);
+                    uint32_t w0, w1, w2, w3;
+                    ptx::ldmatrix_x4(sK + r * Cfg::kRowBytes + ((u ^ (r & 7)) << 4), w0, w1, w2, w3);
+                    w0 ^= 0x80808080u; w1 ^= 0x80808080u; w2 ^= 0x80808080u; w3 ^= 0x80808080u;
+                    // w0: rows 0-7 unit U, w1: rows 8-15 unit U, w2/w3: unit U+1
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        mma16816<QT>(s[nt], s8pair<QT>(w0, 0, 1), s8pair<QT>(w1, 0, 1), s8pair<QT>(w0, 2, 3),
+                                     s8pair<QT>(w1, 2, 3), qf[nt][U][0], qf[nt][U][1]);
+                        mma16816<QT>(s[nt], s8pair<QT>(w2, 0, 1), s8pair<QT>(w3, 0, 1), s8pair<QT>(w2, 2, 3),
+                                     s8pair<QT>(w3, 2, 3), qf[nt][U + 1][0], qf[nt][U + 1][1]);
+                    }
+                }
+            }
+        }
+
+        // ---- online softmax over this chunk (base 2) ----
+        float ks_a = 1.f, ks_b = 1.f, vs_a = 1.f, vs_b = 1.f;
+        if constexpr (Cfg::kInt8) {
+            // Scales were copied as the aligned 4-byte word holding them; the
+            // half is the parity of the element index (slot * Hkv + kvh).  With
+            // page_size a multiple of 16 that parity is kvh's for even Hkv and
+            // (row + kvh)'s for odd Hkv.
+            const uint8_t* sS = ring + (i % STAGES) * Cfg::kStage + 2 * Cfg::kTile;
+            auto scale_at = [&](int base, int row) {
+                const uint32_t w = *reinterpret_cast<const uint32_t*>(sS + base + row * 4);
+                const int odd = ((Hkv & 1) ? (row + kvh) : kvh) & 1;
+                return __half2float(__ushort_as_half(static_cast<unsigned short>(odd ? (w >> 16) : (w & 0xffffu))));
+            };
+            ks_a = scale_at(0, g); ks_b = scale_at(0, g + 8);
+            vs_a = scale_at(64, g); vs_b = scale_at(64, g + 8);
+        }
+        const bool va = tok0 + g < ctx, vb = tok0 + g + 8 < ctx;
+        uint32_t pb[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            float x[4];
+            x[0] = va ? s[nt][0] * (p.scale_log2 * ks_a) : -INFINITY;
+            x[1] = va ? s[nt][1] * (p.scale_log2 * ks_a) : -INFINITY;
+            x[2] = vb ? s[nt][2] * (p.scale_log2 * ks_b) : -INFINITY;
+            x[3] = vb ? s[nt][3] * (p.scale_log2 * ks_b) : -INFINITY;
+            float pr[4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float mx = fmaxf(x[h], x[2 + h]);
+                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+                const float m_new = fmaxf(m[nt][h], mx);   // finite: token tok0 is in the context
+                const float corr = ptx::ex2(m[nt][h] - m_new);
+                m[nt][h] = m_new;
+                pr[h] = ptx::ex2(x[h] - m_new);
+                pr[2 + h] = ptx::ex2(x[2 + h] - m_new);
+                l[nt][h] = l[nt][h] * corr + (pr[h] + pr[2 + h]);
+#pragma unroll
+                for (int dt = 0; dt < Cfg::kDT; ++dt) {
+                    o[nt][dt][h] *= corr;
+                    o[nt][dt][2 + h] *= corr;
+                }
+            }
+            // P^T fragments (B operand of O^T += V^T . P^T) via 8x8 transposes
+            pb[nt][0] = ptx::movmatrix_trans(pack2<QT>(pr[0] * vs_a, pr[1] * vs_a));
+            pb[nt][1] = ptx::movmatrix_trans(pack2<QT>(pr[2] * vs_b, pr[3] * vs_b));
+        }
+
+        // ---- O^T += V^T . P^T ----
+        if constexpr (!Cfg::kInt8) {
+            const int r = (lane & 7) + ((lane >> 4) << 3);
+#pragma unroll
+            for (int dt = 0; dt < Cfg::kDT; ++dt) {
+                const int u = 2 * dt + ((lane >> 3) & 1);
+                uint32_t a0, a1, a2, a3;
+                ptx::ldmatrix_x4_trans(sV + r * Cfg::kRowBytes + ((u ^ (r & 7)) << 4), a0, a1, a2, a3);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma16816<QT>(o[nt][dt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+            }
+        } else {
+            const int r = (lane & 7) + (((lane >> 3) & 1) << 3);
+#pragma unroll
+            for (int U = 0; U < Cfg::kUnits; U += 2) {
+                const int u = U + (lane >> 4);
+                uint32_t w0, w1, w2, w3;
+                ptx::ldmatrix_x4_trans(sV + r * Cfg::kRowBytes + ((u ^ (r & 7)) << 4), w0, w1, w2, w3);
+                w0 ^= 0x80808080u; w1 ^= 0x80808080u; w2 ^= 0x80808080u; w3 ^= 0x80808080u;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    mma16816<QT>(o[nt][U], s8pair<QT>(w0, 0, 2), s8pair<QT>(w0, 1, 3), s8pair<QT>(w1, 0, 2),
+                                 s8pair<QT>(w1, 1, 3), pb[nt][0], pb[nt][1]);
+                    mma16816<QT>(o[nt][U + 1], s8pair<QT>(w2, 0, 2), s8pair<QT>(w2, 1, 3), s8pair<QT>(w3, 0, 2),
+                                 s8pair<QT>(w3, 1, 3), pb[nt][0], pb[nt][1]);
+                }
+            }
+        }
+        __syncwarp();
+    }
+    ptx::cp_async_wait<0>();
+
+    // ---- merge the warps' partial softmax states ----
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float x = l[nt][h];
+            x += __shfl_xor_sync(kFull, x, 4);
+            x += __shfl_xor_sync(kFull, x, 8);
+            x += __shfl_xor_sync(kFull, x, 16);
+            l[nt][h] = x;
+        }
+    __syncthreads();
+    constexpr int NH = 8 * NT;
+    float* sm_m = reinterpret_cast<float*>(smem);
+    float* sm_l = sm_m + WARPS * NH;
+    float* sm_o = sm_l + WARPS * NH;
+    if (g == 0) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                sm_m[warp * NH + nt * 8 + 2 * c + h] = m[nt][h];
+                sm_l[warp * NH + nt * 8 + 2 * c + h] = l[nt][h];
+            }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int n = nt * 8 + 2 * c + h;
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < WARPS; ++w) M = fmaxf(M, sm_m[w * NH + n]);
+            const float f = (m[nt][h] == -INFINITY) ? 0.f : ptx::ex2(m[nt][h] - M);
+            float* dst = sm_o + (warp * NH + n) * HD;
+#pragma unroll
+            for (int dt = 0; dt < Cfg::kDT; ++dt) {
+                const int d_lo = Cfg::kInt8 ? dt * 16 + 2 * g : dt * 16 + g;
+                const int d_hi = Cfg::kInt8 ? d_lo + 1 : d_lo + 8;
+                dst[d_lo] = o[nt][dt][h] * f;
+                dst[d_hi] = o[nt][dt][2 + h] * f;
+            }
+        }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < G * HD; idx += WARPS * 32) {
+        const int n = idx / HD, d = idx % HD;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < WARPS; ++w) M = fmaxf(M, sm_m[w * NH + n]);
+        float L = 0.f, acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < WARPS; ++w) {
+            const float mw = sm_m[w * NH + n];
+            L += (mw == -INFINITY) ? 0.f : sm_l[w * NH + n] * ptx::ex2(mw - M);
+            acc += sm_o[(w * NH + n) * HD + d];
+        }
+        const float val = acc / L;
+        if (nsplit == 1) {
+            out[(head0 + n) * HD + d] = from_float<QT>(val);
+        } else {
+            const size_t row = (head0 + n) * p.max_splits + split;
+            p.o_part[row * HD + d] = val;
+            if (d == 0) p.lse_part[row] = M + __log2f(L);
+        }
+    }
+}
+
+// Merge of the split-KV partials of one (sequence, query head) per warp.
+template <typename QT, int HD>
+__global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gw = blockIdx.x * 4 + warp;
+    if (gw >= p.num_seqs * p.num_q_heads) return;
+    const int b = gw / p.num_q_heads;
+    const int ctx = __ldg(p.context_lens + b);
+    if (ctx <= 0 || ctx > p.max_pages_per_seq * p.page_size) return;
+    const int ns = ceil_div(ceil_div(ctx, kChunk), p.chunks_per_split);
+    if (ns <= 1) return;
+    const float* lse = p.lse_part + static_cast<size_t>(gw) * p.max_splits;
+    const float* op = p.o_part + static_cast<size_t>(gw) * p.max_splits * HD;
+    float M = -INFINITY;
+    for (int s = lane; s < ns; s += 32) M = fmaxf(M, lse[s]);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
+    constexpr int E = HD / 32;
+    float acc[E];
+#pragma unroll
+    for (int j = 0; j < E; ++j) acc[j] = 0.f;
+    float W = 0.f;
+#pragma unroll 4
+    for (int s = 0; s < ns; ++s) {
+        const float w = ptx::ex2(lse[s] - M);
+        W += w;
+        const float* src = op + static_cast<size_t>(s) * HD + lane * E;
+        if constexpr (E == 4) {
+            const float4 v = *reinterpret_cast<const float4*>(src);
+            acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
+        } else {
+#pragma unroll
+            for (int j = 0; j < E; ++j) acc[j] += w * src[j];
+        }
+    }
+    QT* out = static_cast<QT*>(p.out) + static_cast<size_t>(gw) * HD + lane * E;
+    const float inv = 1.f / W;
+#pragma unroll
+    for (int j = 0; j < E; ++j) out[j] = from_float<QT>(acc[j] * inv);
+}
+
+// fp32 pages and queries (small problems; CUDA-core path with exact-ish fp32
+// arithmetic): one warp per query head, lanes across head_dim.
+template <int HD>
+__global__ void __launch_bounds__(128) decode_f32_kernel(const DecodeParams p) {
+    const int kvh = blockIdx.x, b = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int Hq = p.num_q_heads, Hkv = p.num_kv_heads, G = Hq / Hkv, ps = p.page_size;
+    const int ctx = __ldg(p.context_lens + b);
+    if (ctx < 0 || ctx > p.max_pages_per_seq * ps) {
+        if (kvh == 0 && threadIdx.x == 0) record_error(p.status, PKV_ERR_DEVICE_RANGE, ctx);
+        return;
+    }
+    constexpr int E = HD / 32;
+    const float* q = static_cast<const float*>(p.q);
+    const float* kp = static_cast<const float*>(p.k_pages);
+    const float* vp = static_cast<const float*>(p.v_pages);
+    float* out = static_cast<float*>(p.out);
+    const int32_t* bt = p.block_tables + static_cast<size_t>(b) * p.max_pages_per_seq;
+    for (int n = warp; n < G; n += 4) {
+        const size_t h = static_cast<size_t>(b) * Hq + static_cast<size_t>(kvh) * G + n;
+        float qv[E], acc[E];
+#pragma unroll
+        for (int j = 0; j < E; ++j) { qv[j] = q[h * HD + lane + 32 * j]; acc[j] = 0.f; }
+        float mx = -INFINITY, l = 0.f;
+        for (int t = 0; t < ctx; ++t) {
+            const int page = __ldg(bt + t / ps);
+            if (page < 0 || page >= p.num_pages) {
+                if (lane == 0) record_error(p.status, PKV_ERR_DEVICE_RANGE, page);
+                continue;
+            }
+            const size_t row = ((static_cast<size_t>(page) * ps + t % ps) * Hkv + kvh) * HD;
+            float dot = 0.f;
+#pragma unroll
+            for (int j = 0; j < E; ++j) dot = fmaf(qv[j], __ldg(kp + row + lane + 32 * j), dot);
+#pragma unroll
+            for (int off = 16; off; off >>= 1) dot += __shfl_xor_sync(kFull, dot, off);
+            const float x = dot * p.scale_log2;
+            const float m_new = fmaxf(mx, x);
+            const float corr = exp2f(mx - m_new);
+            const float pr = exp2f(x - m_new);
+            l = l * corr + pr;
+#pragma unroll
+            for (int j = 0; j < E; ++j) acc[j] = fmaf(pr, __ldg(vp + row + lane + 32 * j), acc[j] * corr);
+            mx = m_new;
+        }
+#pragma unroll
+        for (int j = 0; j < E; ++j) out[h * HD + lane + 32 * j] = ctx > 0 ? acc[j] / l : 0.f;
+    }
+}
+
+constexpr int kWarps = 4;
+constexpr int kStages = 3;
+
+template <typename QT, typename KVT, int HD, int NT>
+cudaError_t run_mma(const DecodeParams& p, cudaStream_t stream) {
+    using Cfg = DecodeCfg<QT, KVT, HD, NT, kWarps, kStages>;
+    auto kern = decode_mma_kernel<QT, KVT, HD, NT, kWarps, kStages>;
+    cudaError_t e0 = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), Cfg::kSmem);
+    if (e0 != cudaSuccess) return e0;
+    dim3 grid(p.max_splits, p.num_kv_heads, p.num_seqs);
+    kern<<<grid, kWarps * 32, Cfg::kSmem, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || p.max_splits == 1) return e;
+    const int warps = p.num_seqs * p.num_q_heads;
+    decode_combine_kernel<QT, HD><<<ceil_div(warps, 4), 128, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename QT, typename KVT, int HD>
+cudaError_t run_nt(const DecodeParams& p, cudaStream_t stream) {
+    const int G = p.num_q_heads / p.num_kv_heads;
+    if (G <= 8) return run_mma<QT, KVT, HD, 1>(p, stream);
+    return run_mma<QT, KVT, HD, 2>(p, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DecodeParams& p, pkv_dtype q_dtype, pkv_dtype kv_dtype,
+                          cudaStream_t stream) {
+    if (q_dtype == PKV_F32) {
+        dim3 grid(p.num_kv_heads, p.num_seqs);
+        if (p.head_dim == 128) decode_f32_kernel<128><<<grid, 128, 0, stream>>>(p);
+        else decode_f32_kernel<64><<<grid, 128, 0, stream>>>(p);
+        return cudaGetLastError();
+    }
+    const bool bf = q_dtype == PKV_BF16;
+    if (kv_dtype == PKV_I8)
+        return bf ? run_nt<__nv_bfloat16, int8_t, 128>(p, stream) : run_nt<__half, int8_t, 128>(p, stream);
+    if (p.head_dim == 128)
+        return bf ? run_nt<__nv_bfloat16, __nv_bfloat16, 128>(p, stream) : run_nt<__half, __half, 128>(p, stream);
+    return bf ? run_nt<__nv_bfloat16, __nv_bfloat16, 64>(p, stream) : run_nt<__half, __half, 64>(p, stream);
+}
+
+}  // namespace pkv

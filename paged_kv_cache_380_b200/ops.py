@@ -1,0 +1,188 @@
+"""Thin ctypes binding of libpagedkv (argument marshalling only).
+
+Every function here forwards device pointers, sizes and the current torch CUDA
+stream to the C ABI declared in ``include/pagedkv.h``; all work runs in the
+library's CUDA kernels.  There is no fallback: if ``libpagedkv.so`` is missing
+or cannot be loaded, the first call raises.
+
+Tensor arguments are torch CUDA tensors (torch is used only for device memory
+and streams).  bf16 pools may also be passed as int16/uint16 views.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpagedkv.so")
+_lock = threading.Lock()
+_lib = None
+
+PKV_F32, PKV_BF16, PKV_F16, PKV_I8 = 0, 1, 2, 3
+_DT = {torch.float32: PKV_F32, torch.bfloat16: PKV_BF16, torch.float16: PKV_F16, torch.int8: PKV_I8}
+
+# every symbol include/pagedkv.h declares
+EXPORTS = ("pkv_error_string", "pkv_kv_cache_write", "pkv_paged_attention_decode",
+           "pkv_decode_workspace_size", "pkv_decode_plan", "pkv_paged_attention_prefill",
+           "pkv_get_device_status")
+
+
+class PagedKVError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {error_string(code)} (code {code})")
+
+
+def load(path: str = _LIB_PATH):
+    """Load the shared library and declare the C signatures (raises if absent)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise ImportError(f"libpagedkv.so not built at {path}: run "
+                              "`python -m paged_kv_cache_380_b200.build` (needs nvcc)")
+        lib = ctypes.CDLL(path)
+        P, I, I64, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+        lib.pkv_error_string.argtypes = [I]
+        lib.pkv_error_string.restype = ctypes.c_char_p
+        lib.pkv_kv_cache_write.argtypes = [P, P, P, I64, P, P, I, I, I, I64, I, P, P, P, P, P]
+        lib.pkv_kv_cache_write.restype = I
+        lib.pkv_paged_attention_decode.argtypes = [P, P, P, P, P, F, P, I, I, I, I, I, I, I64, I, I,
+                                                   P, P, P, SZ, I, P]
+        lib.pkv_paged_attention_decode.restype = I
+        lib.pkv_decode_workspace_size.argtypes = [I, I, I, I, I, I, I, I]
+        lib.pkv_decode_workspace_size.restype = SZ
+        lib.pkv_decode_plan.argtypes = [I, I, I, I, I, I, I, I, ctypes.POINTER(I), ctypes.POINTER(I)]
+        lib.pkv_decode_plan.restype = I
+        lib.pkv_paged_attention_prefill.argtypes = [P, P, P, P, P, P, I, F, P, I, I, I, I, I, I, I, I,
+                                                    I64, I, P]
+        lib.pkv_paged_attention_prefill.restype = I
+        lib.pkv_get_device_status.argtypes = [P, ctypes.POINTER(I64)]
+        lib.pkv_get_device_status.restype = I
+        _lib = lib
+    return _lib
+
+
+def error_string(code: int) -> str:
+    return load().pkv_error_string(int(code)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise PagedKVError(rc, what)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype in _DT:
+        return _DT[t.dtype]
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def kv_cache_write(k, v, slot_mapping, k_pages, v_pages, *, k_scale=None, v_scale=None,
+                   k_scale_pages=None, v_scale_pages=None, stream=None) -> None:
+    """Scatter new K/V rows ``[T, Hkv, D]`` into pools ``[P, ps, Hkv, D]`` at
+    ``slot_mapping`` (int64 ``[T]``; negative = skip).  INT8 pools also take
+    the per-row fp16 scales ``[T, Hkv]`` and scale pools ``[P, ps, Hkv]``."""
+    _cuda(k, v, slot_mapping, k_pages, v_pages, k_scale, v_scale, k_scale_pages, v_scale_pages)
+    P, ps, Hkv, D = k_pages.shape
+    if slot_mapping.dtype != torch.int64:
+        raise TypeError("slot_mapping must be int64")
+    if k.shape[1:] != (Hkv, D) or v.shape != k.shape or k.dtype != k_pages.dtype:
+        raise ValueError("k/v must be [T, num_kv_heads, head_dim] of the pool's dtype")
+    _check(load().pkv_kv_cache_write(_ptr(k), _ptr(v), _ptr(slot_mapping), k.shape[0], _ptr(k_pages),
+                                     _ptr(v_pages), Hkv, D, ps, P, _dtype_code(k_pages), _ptr(k_scale),
+                                     _ptr(v_scale), _ptr(k_scale_pages), _ptr(v_scale_pages),
+                                     _stream(stream)), "kv_cache_write")
+
+
+def decode_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, page_size, max_pages_per_seq,
+                kv_dtype=torch.bfloat16, num_splits=0):
+    """(partitions per sequence, partition length in tokens) the decode call uses."""
+    s, t = ctypes.c_int(0), ctypes.c_int(0)
+    _check(load().pkv_decode_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, page_size,
+                                  max_pages_per_seq, _DT[kv_dtype], num_splits, ctypes.byref(s),
+                                  ctypes.byref(t)), "decode_plan")
+    return s.value, t.value
+
+
+def decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, page_size, max_pages_per_seq,
+                          kv_dtype=torch.bfloat16, num_splits=0) -> int:
+    return int(load().pkv_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, page_size,
+                                                max_pages_per_seq, _DT[kv_dtype], num_splits))
+
+
+def paged_attention_decode(q, k_pages, v_pages, block_tables, context_lens, scale, out=None, *,
+                           k_scales=None, v_scales=None, workspace=None, num_splits=0, stream=None):
+    """Decode attention: ``q [B, Hq, D]`` against pools ``[P, ps, Hkv, D]``
+    through ``block_tables int32 [B, MP]`` and ``context_lens int32 [B]``.
+    Returns ``out`` (allocated like ``q`` if not given).  A workspace of
+    ``decode_workspace_size(...)`` bytes is allocated with torch when the
+    caller passes none."""
+    _cuda(q, k_pages, v_pages, block_tables, context_lens, k_scales, v_scales, out, workspace)
+    B, Hq, D = q.shape
+    P, ps, Hkv, D2 = k_pages.shape
+    if D2 != D or v_pages.shape != k_pages.shape or block_tables.shape[0] != B:
+        raise ValueError("shape mismatch")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    if out is None:
+        out = torch.empty_like(q)
+    MP = block_tables.shape[1]
+    kv_dt = k_pages.dtype
+    if workspace is None:
+        need = decode_workspace_size(B, Hq, Hkv, D, ps, MP, kv_dt, num_splits)
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _check(load().pkv_paged_attention_decode(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_tables), _ptr(context_lens), float(scale),
+        _ptr(out), B, Hq, Hkv, D, ps, MP, P, _dtype_code(q), _dtype_code(k_pages), _ptr(k_scales),
+        _ptr(v_scales), _ptr(workspace), workspace.numel(), int(num_splits), _stream(stream)),
+        "paged_attention_decode")
+    return out
+
+
+def paged_attention_prefill(q, k_pages, v_pages, block_tables, q_start, context_lens, causal, scale,
+                            out=None, *, max_q_len=None, stream=None):
+    """Chunked prefill: packed ``q [Ttot, Hq, D]``, rows ``q_start[b]..q_start[b+1]-1``
+    of sequence b at positions ``ctx-n..ctx-1``; causal rows see keys up to
+    their own position.  ``max_q_len`` (the longest chunk) sizes the grid;
+    when omitted it is read from ``q_start`` (a device-to-host copy)."""
+    _cuda(q, k_pages, v_pages, block_tables, q_start, context_lens, out)
+    T, Hq, D = q.shape
+    P, ps, Hkv, D2 = k_pages.shape
+    B = context_lens.shape[0]
+    if D2 != D or q_start.shape[0] != B + 1:
+        raise ValueError("shape mismatch")
+    if out is None:
+        out = torch.empty_like(q)
+    if max_q_len is None:
+        max_q_len = int((q_start[1:] - q_start[:-1]).max().item()) if B else 0
+    _check(load().pkv_paged_attention_prefill(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_tables), _ptr(q_start), _ptr(context_lens),
+        1 if causal else 0, float(scale), _ptr(out), B, T, int(max_q_len), Hq, Hkv, D, ps,
+        block_tables.shape[1], P, _dtype_code(q), _stream(stream)), "paged_attention_prefill")
+    return out
+
+
+def device_status(stream=None):
+    """Synchronise the stream; return (code, detail) of the device status word and clear it."""
+    detail = ctypes.c_int64(-1)
+    code = load().pkv_get_device_status(_stream(stream), ctypes.byref(detail))
+    return int(code), int(detail.value)

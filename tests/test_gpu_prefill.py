@@ -1,0 +1,77 @@
+"""GPU parity: causal chunked prefill over a paged cache with a shared prefix,
+against the fp64 oracle (max abs error 2e-2 for bf16/fp16)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import assert_close, assert_status_ok, dev, f64
+from paged_kv_cache_380_b200 import ops
+from paged_kv_cache_380_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def run_prefill(case, causal=True, items=None, tol=2e-2):
+    """Append the chunk's K/V (cache write), then prefill; compare with the oracle."""
+    tag = case.dtype
+    kp, vp = dev(case.k_pages, tag), dev(case.v_pages, tag)
+    ops.kv_cache_write(dev(case.k_new, tag), dev(case.v_new, tag), dev(case.slot_mapping, "i64"), kp, vp)
+    k_host, v_host = case.k_pages.copy(), case.v_pages.copy()
+    oracle.kv_cache_write(case.k_new, case.v_new, case.slot_mapping, k_host, v_host)
+    q = dev(case.q, tag)
+    max_q = int(np.max(np.diff(case.q_start))) if case.batch else 0
+    out = ops.paged_attention_prefill(q, kp, vp, dev(case.block_tables, "i32"), dev(case.q_start, "i32"),
+                                      dev(case.context_lens, "i32"), causal, case.scale, max_q_len=max_q)
+    torch.cuda.synchronize()
+    assert_status_ok()
+    want = oracle.prefill(case.q, tag, k_host, v_host, tag, case.block_tables, case.q_start,
+                          case.context_lens, causal, case.scale, items=items)
+    got = f64(out)
+    got = got.reshape(-1, got.shape[-1])[items] if items is not None else got
+    assert_close(got, want, tol, case.name)
+
+
+def case(idx, chunks, private_prefix=0, shared_prefix=32, Hq=8, Hkv=2, ps=16, dtype="bf16"):
+    return W.prefill_case(name=f"prefill{idx}", config_index=200 + idx, num_seqs=len(chunks),
+                          num_q_heads=Hq, num_kv_heads=Hkv, head_dim=128, page_size=ps, dtype=dtype,
+                          shared_prefix=shared_prefix, chunk_lens=np.array(chunks),
+                          private_prefix=private_prefix)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_ragged_chunks_and_prefixes(causal):
+    # chunks shorter than a tile, exactly a tile, ragged tails; chunks start mid-page
+    run_prefill(case(1, chunks=(1, 5, 64, 130, 200, 128), private_prefix=7), causal=causal)
+
+
+def test_no_prefix():
+    run_prefill(case(2, chunks=(1, 17, 300), shared_prefix=0))
+
+
+def test_long_prefix_short_chunk():
+    run_prefill(case(3, chunks=(3, 1, 70), shared_prefix=1024, private_prefix=100))
+
+
+def test_mha_and_large_pages():
+    run_prefill(case(4, chunks=(90, 257), Hq=4, Hkv=4, ps=256, shared_prefix=256, private_prefix=3))
+
+
+def test_fp16():
+    run_prefill(case(5, chunks=(40, 129), dtype="f16", private_prefix=11))
+
+
+def test_empty_sequence_in_batch():
+    run_prefill(case(6, chunks=(0, 50, 0, 3)))
+
+
+def test_chunked_prefill_shared_prefix_full():
+    """8 x 512 rows after a shared 1024-token prefix; sampled rows checked."""
+    c = W.chunked_prefill_shared_prefix()
+    rng = np.random.default_rng(0)
+    Hq = c.num_q_heads
+    T = c.q.shape[0]
+    items = set(rng.choice(T * Hq, 3000, replace=False).tolist())
+    for t in (0, 1, 127, 128, 255, 511, 512, 1023, 2047, 4095):   # tile edges, sequence edges
+        items |= {t * Hq + h for h in range(Hq)}
+    run_prefill(c, items=np.array(sorted(items)))
