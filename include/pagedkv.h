@@ -93,6 +93,28 @@ int pkv_kv_cache_write(const void* k, const void* v, const int64_t* slot_mapping
                        void* k_scale_pages, void* v_scale_pages, pkv_stream_t stream);
 
 /*
+ * Cache append with INT8 quantisation fused in: each (token, KV head) row of
+ * k and v (head_dim elements of src_dtype: PKV_BF16, PKV_F16 or PKV_F32) is
+ * quantised symmetrically to 8 bits with one fp16 scale per row ([SYS] §3.2
+ * "量化压缩的工程实践" with bits = 8 and one group per row: a = max|x|,
+ * scale = fp16(a / 127) rounded to nearest even, code =
+ * clamp(round_half_even(x / scale), -127, 127) in IEEE fp32; a zero scale or
+ * a NaN element gives code 0) and written to slot slot_mapping[t] of the INT8
+ * pools and of the fp16 scale pools.
+ *
+ *   k, v           [num_tokens][num_kv_heads][head_dim], head_dim 64 or 128
+ *   k_pages, v_pages           int8 [num_pages][page_size][num_kv_heads][head_dim]
+ *   k_scale_pages, v_scale_pages fp16 [num_pages][page_size][num_kv_heads]
+ *   slot_mapping   int64 [num_tokens], as for pkv_kv_cache_write
+ * Codes and scales are bit-identical to the definition above (deterministic).
+ */
+int pkv_kv_cache_write_quant(const void* k, const void* v, pkv_dtype src_dtype,
+                             const int64_t* slot_mapping, int64_t num_tokens, void* k_pages,
+                             void* v_pages, void* k_scale_pages, void* v_scale_pages,
+                             int num_kv_heads, int head_dim, int page_size, int64_t num_pages,
+                             pkv_stream_t stream);
+
+/*
  * Decode attention: one query token per sequence attends all context_lens[b]
  * cached keys of its sequence (no mask; the query is the last token of the
  * context):  out[b][h] = softmax(scale * q[b][h] . K_b^T) V_b  ([KVFA] §2.1,

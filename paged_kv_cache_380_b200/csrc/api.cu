@@ -152,6 +152,26 @@ int pkv_kv_cache_write(const void* k, const void* v, const int64_t* slot_mapping
     return rc;
 }
 
+int pkv_kv_cache_write_quant(const void* k, const void* v, pkv_dtype src_dtype, const int64_t* slot_mapping,
+                             int64_t num_tokens, void* k_pages, void* v_pages, void* k_scale_pages,
+                             void* v_scale_pages, int num_kv_heads, int head_dim, int page_size,
+                             int64_t num_pages, pkv_stream_t stream) {
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || page_size <= 0 || num_pages <= 0)
+        return PKV_ERR_INVALID_ARG;
+    if (src_dtype != PKV_BF16 && src_dtype != PKV_F16 && src_dtype != PKV_F32) return PKV_ERR_UNSUPPORTED;
+    if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return PKV_OK;
+    if (!k || !v || !slot_mapping || !k_pages || !v_pages || !k_scale_pages || !v_scale_pages ||
+        !aligned(slot_mapping, 8) || !aligned(k_scale_pages, 2) || !aligned(v_scale_pages, 2))
+        return PKV_ERR_INVALID_ARG;
+    if (num_tokens > 0xffffffffLL) return PKV_ERR_UNSUPPORTED;
+    DeviceStatus* st = status_ptr();
+    if (!st) return PKV_ERR_CUDA;
+    return from_cuda(launch_kv_quant_scatter(k, v, src_dtype, slot_mapping, num_tokens, num_kv_heads, head_dim,
+                                             k_pages, v_pages, k_scale_pages, v_scale_pages,
+                                             num_pages * page_size, st, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int pkv_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int page_size,
                     int max_pages_per_seq, pkv_dtype kv_dtype, int num_splits, int* splits_out,
                     int* split_tokens_out) {

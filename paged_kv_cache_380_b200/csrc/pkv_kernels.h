@@ -17,6 +17,13 @@ cudaError_t launch_kv_scatter(const void* src_k, const void* src_v, const int64_
                               int64_t num_tokens, void* dst_k, void* dst_v, int64_t row_bytes,
                               int64_t num_slots, DeviceStatus* status, cudaStream_t stream);
 
+// Quantise-on-write: rows of head_dim (64 or 128) elements of src_dtype
+// (bf16/f16/f32) become int8 codes + one fp16 scale per (token, head) row.
+cudaError_t launch_kv_quant_scatter(const void* src_k, const void* src_v, pkv_dtype src_dtype,
+                                    const int64_t* slots, int64_t num_tokens, int num_kv_heads, int head_dim,
+                                    void* k_pages, void* v_pages, void* k_scales, void* v_scales,
+                                    int64_t num_slots, DeviceStatus* status, cudaStream_t stream);
+
 // ---- decode ------------------------------------------------------------------
 struct DecodeParams {
     const void* q;

@@ -1,16 +1,39 @@
-// Chunked-prefill attention over a paged KV cache (causal, bottom-right).
+// Chunked-prefill attention over a paged KV cache on the 5th-generation tensor
+// cores (tcgen05 + TMEM), operands staged by TMA.
 //
-// Query rows q_start[b] .. q_start[b+1]-1 of sequence b sit at absolute
-// positions ctx-n .. ctx-1; row r attends keys 0 .. ctx-n+r (causal) or all
-// ctx keys.  FlashAttention-style tiling ("Flash Attention与Paged KV Cache优化
-// 大模型计算效率" §2.1: tiles of Q and K/V staged on chip, softmax computed
-// per tile; "大模型推理优化实战：KV Cache + Flash Attention，让 Token 生成快 3 倍",
-// "Flash Attention 的分块计算原理": online max/sum with rescaling), K/V tiles
-// gathered through the block table.
+// What is computed: query rows q_start[b] .. q_start[b+1]-1 of sequence b sit
+// at absolute positions ctx-n .. ctx-1 (bottom-right alignment: the chunk
+// follows the cached prefix); row r attends keys 0 .. ctx-n+r when causal,
+// else all ctx keys; out = softmax(scale * q K^T) V.  FlashAttention-style
+// tiling ("Flash Attention与Paged KV Cache优化大模型计算效率" §2.1: Q and K/V
+// tiles staged on chip, 128x128 tiles; §4.1: prompt processing with
+// FlashAttention) with the online softmax of "大模型推理优化实战：KV Cache +
+// Flash Attention，让 Token 生成快 3 倍" ("Flash Attention 的分块计算原理"),
+// K/V read page by page through the block table.
 //
-// This version runs the two contractions with warp-level mma.sync (16 query
-// rows per warp, 64-key tiles, cp.async double buffering).
+// B200 design, one CTA per (128-row query tile, query head, sequence):
+//  * warp 0 = TMA producer: Q tile once (two 64-column SW128 boxes), then per
+//    128-key tile one 16-row box per page group and 64-column half for K and
+//    for V, into rings of 3 K stages and 2 V stages (mbarrier expect_tx).
+//  * warp 1 = MMA issuer (one thread): S_j = Q K_j^T (M=128, N=128, K=128,
+//    bf16 -> fp32 in TMEM, triple-buffered) and O += P_j V_j with P read from
+//    TMEM (the TS form) and V as an MN-major operand; tcgen05.commit signals
+//    S ready, the K stage free, O updated and the V stage free.
+//  * warps 2-5 = softmax: one TMEM lane (query row) per thread; tcgen05.ld of
+//    the S row, masking, row max, exp2, row sum, P packed to bf16 pairs and
+//    tcgen05.st back over the S columns.  The accumulator is rescaled only
+//    when a row's running max grows by more than 2^8 (P <= 256 otherwise),
+//    which keeps O's TMEM round trip off most tiles; the final division by
+//    the row sum makes any consistent reference max exact.
+//  * Heaviest (longest causal) query tiles are launched first.
+//  * Every mbarrier wait is bounded; on time-out the CTA records
+//    PKV_ERR_DEVICE_TIMEOUT, raises an abort flag so every role leaves its
+//    loop, waits (bounded) for its own async work and frees TMEM.
+#include <cuda.h>
+
 #include <cmath>
+#include <cstring>
+#include <mutex>
 #include <type_traits>
 
 #include "pkv_kernels.h"
@@ -19,211 +42,391 @@
 namespace pkv {
 namespace {
 
-constexpr unsigned kFull = 0xffffffffu;
-constexpr int BM = 64, BN = 64, HD = 128, kRowB = HD * 2, kUnits = kRowB / 16;
-constexpr int kThreads = 128;
-constexpr int kTileB = BN * kRowB;   // one K or V tile
-constexpr int kSmem = BM * kRowB + 4 * kTileB;
+constexpr int BM = 128, BN = 128, HD = 128;
+constexpr int KST = 3, VST = 2, NSB = 3;        // K stages, V stages, S/P TMEM buffers
+constexpr int kThreads = 192;
+constexpr int kAtom = BN * 128;                 // one 64-column SW128 half of a 128-row tile
+constexpr int kTile = 2 * kAtom;                // 32 KB
+constexpr int kSmemQ = 0;
+constexpr int kSmemK = kSmemQ + kTile;
+constexpr int kSmemV = kSmemK + KST * kTile;
+constexpr int kSmemBar = kSmemV + VST * kTile;
+constexpr int kNumBars = 1 + 2 * KST + 2 * VST + 3 * NSB + 1;
+constexpr int kSmemBytes = kSmemBar + kNumBars * 8 + 16 + 1024;   // + TMEM addr, abort flag, alignment
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kOCol = NSB * 128;           // O accumulator columns 384..511
+constexpr float kRescaleThreshold = 8.0f;       // log2 units: rescale when the max grows by > 2^8
 
-template <typename T>
-__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
-    if constexpr (std::is_same<T, __nv_bfloat16>::value)
-        ptx::mma_bf16_16816(d, a0, a1, a2, a3, b0, b1);
-    else
-        ptx::mma_f16_16816(d, a0, a1, a2, a3, b0, b1);
+// sm_100 shared-memory matrix descriptor: start, leading and stride byte
+// offsets (>> 4), version 1, SWIZZLE_128B layout.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) |
+           (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+           (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
-__device__ __forceinline__ uint32_t swz(int r, int u) { return r * kRowB + ((u ^ (r & 7)) << 4); }
+// Instruction descriptor, kind::f16: D fp32, A/B bf16 (fmt 1) or f16 (fmt 0),
+// N and M as given, B K-major (0) or MN-major (1).
+template <typename T>
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int b_mn_major) {
+    constexpr uint32_t fmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
+    return (1u << 4) | (fmt << 7) | (fmt << 10) | (static_cast<uint32_t>(b_mn_major) << 16) |
+           (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// mbarrier addresses, all in one array after the tiles.
+struct Bars {
+    uint32_t base;
+    __device__ __forceinline__ uint32_t q_full() const { return base; }
+    __device__ __forceinline__ uint32_t k_full(int i) const { return base + 8 * (1 + i); }
+    __device__ __forceinline__ uint32_t k_empty(int i) const { return base + 8 * (1 + KST + i); }
+    __device__ __forceinline__ uint32_t v_full(int i) const { return base + 8 * (1 + 2 * KST + i); }
+    __device__ __forceinline__ uint32_t v_empty(int i) const { return base + 8 * (1 + 2 * KST + VST + i); }
+    __device__ __forceinline__ uint32_t s_full(int i) const { return base + 8 * (1 + 2 * KST + 2 * VST + i); }
+    __device__ __forceinline__ uint32_t p_full(int i) const { return base + 8 * (1 + 2 * KST + 2 * VST + NSB + i); }
+    __device__ __forceinline__ uint32_t pv_done(int i) const { return base + 8 * (1 + 2 * KST + 2 * VST + 2 * NSB + i); }
+    __device__ __forceinline__ uint32_t mma_done() const { return base + 8 * (1 + 2 * KST + 2 * VST + 3 * NSB); }
+};
+
+// Bounded wait that also gives up as soon as another role raised the abort flag.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         DeviceStatus* st) {
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+    }
+    *abort_flag = 1;
+    record_error(st, PKV_ERR_DEVICE_TIMEOUT, static_cast<long long>(bar));
+    return false;
+}
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads) prefill_mma_kernel(const PrefillParams p) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
-    const int mt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = ptx::smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    const int num_qt = gridDim.z;
+    const int qt = num_qt - 1 - static_cast<int>(blockIdx.z);   // heaviest tiles first
+    const int h = blockIdx.x, b = blockIdx.y;
     const int Hq = p.num_q_heads, Hkv = p.num_kv_heads, kvh = h / (Hq / Hkv), ps = p.page_size;
     const int q0 = __ldg(p.q_start + b), n = __ldg(p.q_start + b + 1) - q0;
     const int ctx = __ldg(p.context_lens + b);
-    const int r0 = mt * BM;
-    if (r0 >= n) return;
-    if (n > ctx || ctx > p.max_pages_per_seq * ps) {
-        if (mt == 0 && h == 0 && tid == 0) record_error(p.status, PKV_ERR_DEVICE_RANGE, ctx);
+    const int r0 = qt * BM;
+    if (r0 >= n) return;                                        // whole CTA, before any barrier
+    if (n > ctx || ctx > p.max_pages_per_seq * ps || q0 < 0 || q0 + n > p.total_q) {
+        if (threadIdx.x == 0) record_error(p.status, PKV_ERR_DEVICE_RANGE, ctx);
         return;
     }
     const int last_row = min(r0 + BM, n) - 1;
     const int max_key = p.causal ? ctx - n + last_row : ctx - 1;
     const int n_tiles = max_key / BN + 1;
+    const int min_lim = p.causal ? ctx - n + r0 : ctx - 1;      // every row of the tile sees keys <= this
 
-    const uint32_t sQ = ptx::smem_u32(smem);
-    const uint32_t sKV = sQ + BM * kRowB;   // [buf][K|V]
-    const uint8_t* kpool = static_cast<const uint8_t*>(p.k_pages);
-    const uint8_t* vpool = static_cast<const uint8_t*>(p.v_pages);
-    const int32_t* bt = p.block_tables + static_cast<size_t>(b) * p.max_pages_per_seq;
+    const Bars bars{sbase + kSmemBar};
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kSmemBar + kNumBars * 8);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSmemBar + kNumBars * 8 + 8);
 
-    // Q tile (rows past the chunk are zero-filled)
-    {
-        const uint8_t* q = static_cast<const uint8_t*>(p.q);
-        for (int x = tid; x < BM * kUnits; x += kThreads) {
-            const int r = x / kUnits, u = x % kUnits;
-            const bool ok = r0 + r < n;
-            const size_t off = (static_cast<size_t>(q0 + r0 + r) * Hq + h) * kRowB + u * 16;
-            ptx::cp_async16(sQ + swz(r, u), ok ? q + off : q, ok ? 16u : 0u);
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(bars.q_full(), 1);
+        for (int i = 0; i < KST; ++i) { ptx::mbar_init(bars.k_full(i), 1); ptx::mbar_init(bars.k_empty(i), 1); }
+        for (int i = 0; i < VST; ++i) { ptx::mbar_init(bars.v_full(i), 1); ptx::mbar_init(bars.v_empty(i), 1); }
+        for (int i = 0; i < NSB; ++i) {
+            ptx::mbar_init(bars.s_full(i), 1);
+            ptx::mbar_init(bars.p_full(i), 128);
+            ptx::mbar_init(bars.pv_done(i), 1);
         }
+        ptx::mbar_init(bars.mma_done(), 1);
+        *abort_flag = 0;
+        ptx::fence_mbarrier_init();
     }
-    auto load_tile = [&](int j) {
-        const uint32_t sK = sKV + (j & 1) * 2 * kTileB, sV = sK + kTileB;
-        for (int x = tid; x < BN * kUnits; x += kThreads) {
-            const int r = x / kUnits, u = x % kUnits;
-            const int key = j * BN + r;
-            bool ok = key < ctx;
-            int page = 0;
-            if (ok) {
-                page = __ldg(bt + key / ps);
-                if (page < 0 || page >= p.num_pages) {
-                    if (u == 0) record_error(p.status, PKV_ERR_DEVICE_RANGE, page);
-                    ok = false;
+    if (warp == 1) {
+        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------ TMA producer ------------------------------
+        const int32_t* bt = p.block_tables + static_cast<size_t>(b) * p.max_pages_per_seq;
+        if (lane == 0) {
+            ptx::prefetch_tmap(&tm_q);
+            ptx::prefetch_tmap(&tm_k);
+            ptx::prefetch_tmap(&tm_v);
+            ptx::mbar_arrive_expect_tx(bars.q_full(), kTile);
+            ptx::tma_load_3d(sbase + kSmemQ, &tm_q, bars.q_full(), 0, h, q0 + r0);
+            ptx::tma_load_3d(sbase + kSmemQ + kAtom, &tm_q, bars.q_full(), 64, h, q0 + r0);
+        }
+        bool ok = true;
+        for (int t = 0; t < n_tiles && ok; ++t) {
+            // lane g < 8 resolves the page of 16-key group g of this tile
+            const int key0 = t * BN + 16 * (lane & 7);
+            int row = -1;
+            if (lane < 8 && key0 < ctx) {
+                const int page = __ldg(bt + key0 / ps);
+                if (page >= 0 && page < p.num_pages) row = page * ps + key0 % ps;
+                else record_error(p.status, PKV_ERR_DEVICE_RANGE, page);
+            }
+            const unsigned valid = __ballot_sync(0xffffffffu, row >= 0) & 0xffu;
+            const uint32_t bytes = __popc(valid) * 16 * 128 * 2;
+            const int ks = t % KST, vs = t % VST;
+            if (t >= KST) ok = wait_bar(bars.k_empty(ks), ((t / KST) - 1) & 1, abort_flag, p.status);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
+            if (lane == 0) ptx::mbar_arrive_expect_tx(bars.k_full(ks), bytes);
+            __syncwarp();
+            if (row >= 0) {
+                const uint32_t dst = sbase + kSmemK + ks * kTile + (lane & 7) * 2048;
+                ptx::tma_load_3d(dst, &tm_k, bars.k_full(ks), 0, kvh, row);
+                ptx::tma_load_3d(dst + kAtom, &tm_k, bars.k_full(ks), 64, kvh, row);
+            }
+            if (t >= VST) ok = wait_bar(bars.v_empty(vs), ((t / VST) - 1) & 1, abort_flag, p.status);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) break;
+            if (lane == 0) ptx::mbar_arrive_expect_tx(bars.v_full(vs), bytes);
+            __syncwarp();
+            if (row >= 0) {
+                const uint32_t dst = sbase + kSmemV + vs * kTile + (lane & 7) * 2048;
+                ptx::tma_load_3d(dst, &tm_v, bars.v_full(vs), 0, kvh, row);
+                ptx::tma_load_3d(dst + kAtom, &tm_v, bars.v_full(vs), 64, kvh, row);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------ MMA issuer ------------------------------
+        if (lane == 0) {
+            constexpr uint32_t id_s = idesc_f16<T>(BM, BN, 0);
+            constexpr uint32_t id_o = idesc_f16<T>(BM, HD, 1);
+            bool ok = wait_bar(bars.q_full(), 0, abort_flag, p.status);
+            auto issue_pv = [&](int i) {
+                const int bi = i % NSB, vs = i % VST;
+                if (!wait_bar(bars.p_full(bi), (i / NSB) & 1, abort_flag, p.status)) return false;
+                if (!wait_bar(bars.v_full(vs), (i / VST) & 1, abort_flag, p.status)) return false;
+                ptx::tc_fence_after();
+                const uint32_t vbase = sbase + kSmemV + vs * kTile;
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk)
+                    ptx::tc_mma_ts(tmem + kOCol, tmem + bi * 128 + kk * 8,
+                                   sdesc(vbase + kk * 2048, kAtom, 1024), id_o, (i > 0 || kk > 0) ? 1u : 0u);
+                ptx::tc_commit(bars.pv_done(bi));
+                ptx::tc_commit(bars.v_empty(vs));
+                return true;
+            };
+            for (int j = 0; j < n_tiles && ok; ++j) {
+                const int ks = j % KST, bj = j % NSB;
+                ok = wait_bar(bars.k_full(ks), (j / KST) & 1, abort_flag, p.status);
+                if (ok && j >= NSB) ok = wait_bar(bars.pv_done(bj), ((j / NSB) - 1) & 1, abort_flag, p.status);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                const uint32_t kbase = sbase + kSmemK + ks * kTile;
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
+                    ptx::tc_mma_ss(tmem + bj * 128, sdesc(sbase + kSmemQ + off, 16, 1024),
+                                   sdesc(kbase + off, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+                }
+                ptx::tc_commit(bars.s_full(bj));
+                ptx::tc_commit(bars.k_empty(ks));
+                if (j >= 1) ok = issue_pv(j - 1);
+            }
+            if (ok) issue_pv(n_tiles - 1);
+            // drain: every tcgen05 op issued by this thread completes before TMEM is freed
+            ptx::tc_commit(bars.mma_done());
+            ptx::mbar_wait(bars.mma_done(), 0, kSpinLimit);
+        }
+    } else {
+        // ------------------------------ softmax + epilogue ------------------------------
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;                        // TMEM lane == tile row
+        const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        const int lim = min(p.causal ? ctx - n + r0 + row : ctx - 1, ctx - 1);
+        const float sl2 = p.scale_log2;
+        float m_ref = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n_tiles; ++j) {
+            const int bj = j % NSB;
+            ok = wait_bar(bars.s_full(bj), (j / NSB) & 1, abort_flag, p.status);
+            if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+            ptx::tc_fence_after();
+            float x[BN];
+#pragma unroll
+            for (int c4 = 0; c4 < BN / 32; ++c4) {
+                uint32_t r[32];
+                ptx::tmem_ld32(trow + bj * 128 + c4 * 32, r);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) x[c4 * 32 + i] = __uint_as_float(r[i]);
+            }
+            ptx::tc_wait_ld();
+            const bool need_mask = j * BN + BN - 1 > min_lim;
+            float mt = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < BN; ++c) {
+                float v = x[c] * sl2;
+                if (need_mask && j * BN + c > lim) v = -INFINITY;
+                x[c] = v;
+                mt = fmaxf(mt, v);
+            }
+            if (j == 0) {
+                m_ref = mt;                                         // finite: key 0 is always visible
+            } else {
+                const bool want = mt > m_ref + kRescaleThreshold;
+                if (__any_sync(0xffffffffu, want)) {
+                    const float m_new = fmaxf(m_ref, mt);
+                    const float corr = ptx::ex2(m_ref - m_new);
+                    l *= corr;
+                    m_ref = m_new;
+                    const int pj = j - 1;
+                    ok = wait_bar(bars.pv_done(pj % NSB), (pj / NSB) & 1, abort_flag, p.status);
+                    if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+                    ptx::tc_fence_after();
+#pragma unroll
+                    for (int c4 = 0; c4 < HD / 32; ++c4) {
+                        uint32_t r[32];
+                        ptx::tmem_ld32(trow + kOCol + c4 * 32, r);
+                        ptx::tc_wait_ld();
+                        uint32_t w0[16], w1[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            w0[i] = __float_as_uint(__uint_as_float(r[i]) * corr);
+                            w1[i] = __float_as_uint(__uint_as_float(r[16 + i]) * corr);
+                        }
+                        ptx::tmem_st16(trow + kOCol + c4 * 32, w0);
+                        ptx::tmem_st16(trow + kOCol + c4 * 32 + 16, w1);
+                    }
+                    ptx::tc_wait_st();
                 }
             }
-            const size_t off = ((static_cast<size_t>(page) * ps + key % ps) * Hkv + kvh) * kRowB + u * 16;
-            ptx::cp_async16(sK + swz(r, u), ok ? kpool + off : kpool, ok ? 16u : 0u);
-            ptx::cp_async16(sV + swz(r, u), ok ? vpool + off : vpool, ok ? 16u : 0u);
+            float rs = 0.f;
+#pragma unroll
+            for (int c16 = 0; c16 < BN / 32; ++c16) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float a = ptx::ex2(x[c16 * 32 + 2 * i] - m_ref);
+                    const float bb = ptx::ex2(x[c16 * 32 + 2 * i + 1] - m_ref);
+                    rs += a + bb;
+                    pk[i] = pack2<T>(a, bb);
+                }
+                ptx::tmem_st16(trow + bj * 128 + c16 * 16, pk);
+            }
+            l += rs;
+            ptx::tc_wait_st();
+            if (j == n_tiles - 1 && ctx < (j + 1) * BN) {
+                // V rows past the context (tail of the last page, or never loaded) must be
+                // finite zeros: P is 0 there but 0 * NaN would poison O.
+                const int vs = j % VST;
+                ok = wait_bar(bars.v_full(vs), (j / VST) & 1, abort_flag, p.status);
+                if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+                const int first = ctx - j * BN;                     // first invalid row of the tile
+                uint4* vt = reinterpret_cast<uint4*>(smem + kSmemV + vs * kTile);
+                const int tid = threadIdx.x - 64;
+                for (int idx = tid; idx < 2 * (BN - first) * 8; idx += 128) {
+                    const int half = idx / ((BN - first) * 8), rem = idx % ((BN - first) * 8);
+                    vt[(half * kAtom + (first + rem / 8) * 128) / 16 + rem % 8] = make_uint4(0, 0, 0, 0);
+                }
+                ptx::fence_proxy_async_smem();
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(bars.p_full(bj));
         }
-    };
-    load_tile(0);
-    ptx::cp_async_commit();
-
-    uint32_t qa[HD / 16][4];
-    float o[HD / 8][4];
-#pragma unroll
-    for (int dt = 0; dt < HD / 8; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
-    float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
-    const int row_a = r0 + warp * 16 + g, row_b = row_a + 8;
-    const int lim_a = p.causal ? ctx - n + row_a : ctx - 1;
-    const int lim_b = p.causal ? ctx - n + row_b : ctx - 1;
-
-    for (int j = 0; j < n_tiles; ++j) {
-        if (j + 1 < n_tiles) {
-            load_tile(j + 1);
-            ptx::cp_async_commit();
-            ptx::cp_async_wait<1>();
-        } else {
-            ptx::cp_async_wait<0>();
+        // epilogue: O / l -> out
+        if (ok) {
+            const int pj = n_tiles - 1;
+            ok = wait_bar(bars.pv_done(pj % NSB), (pj / NSB) & 1, abort_flag, p.status);
         }
-        __syncthreads();
-        if (j == 0) {
-            const int r = warp * 16 + (lane & 15);
+        if (__all_sync(0xffffffffu, ok)) {
+            ptx::tc_fence_after();
+            const float inv = 1.f / l;
+            const bool store = r0 + row < n;
+            T* out = static_cast<T*>(p.out) + (static_cast<size_t>(q0 + r0 + row) * Hq + h) * HD;
 #pragma unroll
-            for (int kk = 0; kk < HD / 16; ++kk)
-                ptx::ldmatrix_x4(sQ + swz(r, 2 * kk + (lane >> 4)), qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
-        }
-        const uint32_t sK = sKV + (j & 1) * 2 * kTileB, sV = sK + kTileB;
-
-        float s[BN / 8][4];
+            for (int c4 = 0; c4 < HD / 32; ++c4) {
+                uint32_t r[32];
+                ptx::tmem_ld32(trow + kOCol + c4 * 32, r);
+                ptx::tc_wait_ld();
+                uint32_t w[16];
 #pragma unroll
-        for (int nt = 0; nt < BN / 8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+                for (int i = 0; i < 16; ++i)
+                    w[i] = pack2<T>(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+                if (store) {
+                    uint4* dst = reinterpret_cast<uint4*>(out + c4 * 32);
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-#pragma unroll
-            for (int np = 0; np < BN / 16; ++np) {
-                const int r = np * 16 + (lane & 7) + ((lane >> 4) << 3);
-                const int u = 2 * kk + ((lane >> 3) & 1);
-                uint32_t b0, b1, b2, b3;
-                ptx::ldmatrix_x4(sK + swz(r, u), b0, b1, b2, b3);
-                mma16816<T>(s[2 * np], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b0, b1);
-                mma16816<T>(s[2 * np + 1], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b2, b3);
+                    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                }
             }
         }
-        // mask + online softmax (rows row_a, row_b)
-        float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-        for (int nt = 0; nt < BN / 8; ++nt) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int key = j * BN + nt * 8 + 2 * c + (e & 1);
-                const int lim = (e < 2) ? lim_a : lim_b;
-                s[nt][e] = key <= lim ? s[nt][e] * p.scale_log2 : -INFINITY;
-                mx[e >> 1] = fmaxf(mx[e >> 1], s[nt][e]);
-            }
-        }
-        float corr[2];
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            mx[i] = fmaxf(mx[i], __shfl_xor_sync(kFull, mx[i], 1));
-            mx[i] = fmaxf(mx[i], __shfl_xor_sync(kFull, mx[i], 2));
-            const float m_new = fmaxf(m_r[i], mx[i]);
-            // a row whose keys are all masked so far keeps m = -inf: use 0 as its shift
-            const float shift = m_new == -INFINITY ? 0.f : m_new;
-            corr[i] = ptx::ex2(m_r[i] - shift);
-            m_r[i] = m_new;
-            mx[i] = shift;
-        }
-        float rs[2] = {0.f, 0.f};
-#pragma unroll
-        for (int nt = 0; nt < BN / 8; ++nt) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                s[nt][e] = ptx::ex2(s[nt][e] - mx[e >> 1]);
-                rs[e >> 1] += s[nt][e];
-            }
-        }
-        l_r[0] = l_r[0] * corr[0] + rs[0];
-        l_r[1] = l_r[1] * corr[1] + rs[1];
-#pragma unroll
-        for (int dt = 0; dt < HD / 8; ++dt) {
-            o[dt][0] *= corr[0]; o[dt][1] *= corr[0];
-            o[dt][2] *= corr[1]; o[dt][3] *= corr[1];
-        }
-        // O += P V
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint32_t a0 = pack2<T>(s[2 * kk][0], s[2 * kk][1]);
-            const uint32_t a1 = pack2<T>(s[2 * kk][2], s[2 * kk][3]);
-            const uint32_t a2 = pack2<T>(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-            const uint32_t a3 = pack2<T>(s[2 * kk + 1][2], s[2 * kk + 1][3]);
-#pragma unroll
-            for (int dp = 0; dp < HD / 16; ++dp) {
-                const int r = kk * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
-                const int u = 2 * dp + (lane >> 4);
-                uint32_t b0, b1, b2, b3;
-                ptx::ldmatrix_x4_trans(sV + swz(r, u), b0, b1, b2, b3);
-                mma16816<T>(o[2 * dp], a0, a1, a2, a3, b0, b1);
-                mma16816<T>(o[2 * dp + 1], a0, a1, a2, a3, b2, b3);
-            }
-        }
-        __syncthreads();
     }
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        l_r[i] += __shfl_xor_sync(kFull, l_r[i], 1);
-        l_r[i] += __shfl_xor_sync(kFull, l_r[i], 2);
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0 && lane == 0 && *abort_flag) {
+        // let in-flight TMA writes land before the shared memory is handed to another CTA
+        for (int t = 0; t < KST; ++t) ptx::mbar_wait(bars.k_full(t), 0, kSpinLimit >> 4);
     }
-    T* out = static_cast<T*>(p.out);
-    const float inv_a = 1.f / l_r[0], inv_b = 1.f / l_r[1];
-#pragma unroll
-    for (int dt = 0; dt < HD / 8; ++dt) {
-        const int d = dt * 8 + 2 * c;
-        if (row_a < n)
-            *reinterpret_cast<uint32_t*>(out + (static_cast<size_t>(q0 + row_a) * Hq + h) * HD + d) =
-                pack2<T>(o[dt][0] * inv_a, o[dt][1] * inv_a);
-        if (row_b < n)
-            *reinterpret_cast<uint32_t*>(out + (static_cast<size_t>(q0 + row_b) * Hq + h) * HD + d) =
-                pack2<T>(o[dt][2] * inv_b, o[dt][3] * inv_b);
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, kTmemCols);
     }
+}
+
+// ---- host: tensor maps through the driver entry point -------------------------
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encoder() {
+    static EncodeTiled fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return static_cast<EncodeTiled>(nullptr);
+        return reinterpret_cast<EncodeTiled>(f);
+    }();
+    return fn;
+}
+
+// 3-D map over a [rows][heads][128] tensor of 16-bit elements, box {64, 1, box_rows}, SW128.
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t heads, uint64_t rows,
+              uint32_t box_rows) {
+    EncodeTiled enc = encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {HD, heads, rows};
+    const cuuint64_t strides[2] = {HD * 2, heads * HD * 2};
+    const cuuint32_t box[3] = {64, 1, box_rows};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <typename T>
 cudaError_t run(const PrefillParams& p, cudaStream_t stream) {
-    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(prefill_mma_kernel<T>), kSmem);
+    const CUtensorMapDataType dt =
+        std::is_same<T, __nv_bfloat16>::value ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    CUtensorMap tq, tk, tv;
+    const uint64_t pool_rows = static_cast<uint64_t>(p.num_pages) * p.page_size;
+    if (!make_map(&tq, p.q, dt, p.num_q_heads, p.total_q, BM) ||
+        !make_map(&tk, p.k_pages, dt, p.num_kv_heads, pool_rows, 16) ||
+        !make_map(&tv, p.v_pages, dt, p.num_kv_heads, pool_rows, 16))
+        return cudaErrorInvalidValue;
+    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(prefill_tc_kernel<T>), kSmemBytes);
     if (e != cudaSuccess) return e;
-    dim3 grid(ceil_div(p.max_q_len, BM), p.num_q_heads, p.num_seqs);
-    prefill_mma_kernel<T><<<grid, kThreads, kSmem, stream>>>(p);
+    dim3 grid(p.num_q_heads, p.num_seqs, ceil_div(p.max_q_len, BM));
+    prefill_tc_kernel<T><<<grid, kThreads, kSmemBytes, stream>>>(p, tq, tk, tv);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_prefill(const PrefillParams& p, pkv_dtype dtype, cudaStream_t stream) {
-    if (p.max_q_len <= 0 || p.num_seqs <= 0) return cudaSuccess;
+    if (p.max_q_len <= 0 || p.num_seqs <= 0 || p.total_q <= 0) return cudaSuccess;
     return dtype == PKV_BF16 ? run<__nv_bfloat16>(p, stream) : run<__half>(p, stream);
 }
 

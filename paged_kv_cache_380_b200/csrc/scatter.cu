@@ -81,7 +81,88 @@ int sm_count() {
     return n;
 }
 
+// Quantise-on-write: one warp per (token, KV head, K or V) row.  Symmetric
+// 8-bit quantisation of "LLM推理系统优化：KV缓存管理与动态批处理技术" §3.2 with one
+// group per row: a = max|x| (NaN ignored), scale = fp16(a / 127) rounded to
+// nearest even, code = clamp(rint(x / scale), -127, 127) with the division in
+// IEEE fp32 and ties to even; a zero scale (or a NaN element) gives code 0.
+template <typename T, int E>
+__global__ void __launch_bounds__(256)
+kv_quant_scatter_kernel(const T* __restrict__ src_k, const T* __restrict__ src_v, const int64_t* __restrict__ slots,
+                        uint32_t num_tokens, int num_kv_heads, int8_t* __restrict__ kp, int8_t* __restrict__ vp,
+                        __half* __restrict__ ks, __half* __restrict__ vs, int64_t num_slots, DeviceStatus* status) {
+    constexpr int D = 32 * E;
+    const uint64_t rows = static_cast<uint64_t>(num_tokens) * num_kv_heads * 2;
+    const int lane = threadIdx.x & 31;
+    const uint64_t warps = static_cast<uint64_t>(gridDim.x) * (blockDim.x >> 5);
+    for (uint64_t w = (static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; w < rows; w += warps) {
+        const bool is_v = w & 1;
+        const uint64_t th = w >> 1;                      // token * num_kv_heads + head
+        const uint32_t t = static_cast<uint32_t>(th / num_kv_heads);
+        const int head = static_cast<int>(th - static_cast<uint64_t>(t) * num_kv_heads);
+        const int64_t s = __ldg(slots + t);
+        if (s < 0) continue;
+        if (s >= num_slots) {
+            if (lane == 0 && head == 0 && !is_v) record_error(status, PKV_ERR_DEVICE_RANGE, s);
+            continue;
+        }
+        const T* src = (is_v ? src_v : src_k) + th * D + lane * E;
+        float x[E];
+#pragma unroll
+        for (int i = 0; i < E; ++i) x[i] = static_cast<float>(src[i]);
+        float a = 0.f;
+#pragma unroll
+        for (int i = 0; i < E; ++i) a = fmaxf(a, fabsf(x[i]));
+#pragma unroll
+        for (int off = 16; off; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+        const __half s16 = __float2half_rn(__fdiv_rn(a, 127.f));
+        const float sc = __half2float(s16);
+        int8_t q[E];
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            float r = sc != 0.f ? rintf(__fdiv_rn(x[i], sc)) : 0.f;
+            if (r != r) r = 0.f;
+            q[i] = static_cast<int8_t>(fminf(fmaxf(r, -127.f), 127.f));
+        }
+        const uint64_t row = static_cast<uint64_t>(s) * num_kv_heads + head;
+        int8_t* dst = (is_v ? vp : kp) + row * D + lane * E;
+#pragma unroll
+        for (int i = 0; i < E; ++i) dst[i] = q[i];
+        if (lane == 0) (is_v ? vs : ks)[row] = s16;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_kv_quant_scatter(const void* src_k, const void* src_v, pkv_dtype src_dtype,
+                                    const int64_t* slots, int64_t num_tokens, int num_kv_heads, int head_dim,
+                                    void* k_pages, void* v_pages, void* k_scales, void* v_scales,
+                                    int64_t num_slots, DeviceStatus* status, cudaStream_t stream) {
+    if (num_tokens == 0) return cudaSuccess;
+    const uint64_t rows = static_cast<uint64_t>(num_tokens) * num_kv_heads * 2;
+    const uint64_t want = (rows + 7) / 8;
+    const uint64_t cap = static_cast<uint64_t>(sm_count()) * 16;
+    const unsigned blocks = static_cast<unsigned>(want < cap ? want : cap);
+    auto* kp = static_cast<int8_t*>(k_pages);
+    auto* vp = static_cast<int8_t*>(v_pages);
+    auto* ks = static_cast<__half*>(k_scales);
+    auto* vs = static_cast<__half*>(v_scales);
+    const uint32_t T = static_cast<uint32_t>(num_tokens);
+#define PKV_QUANT_LAUNCH(TYPE, E)                                                                         \
+    kv_quant_scatter_kernel<TYPE, E><<<blocks, 256, 0, stream>>>(static_cast<const TYPE*>(src_k),          \
+                                                                 static_cast<const TYPE*>(src_v), slots, T, \
+                                                                 num_kv_heads, kp, vp, ks, vs, num_slots, status)
+    const int E = head_dim / 32;
+    if (src_dtype == PKV_BF16) {
+        if (E == 4) PKV_QUANT_LAUNCH(__nv_bfloat16, 4); else PKV_QUANT_LAUNCH(__nv_bfloat16, 2);
+    } else if (src_dtype == PKV_F16) {
+        if (E == 4) PKV_QUANT_LAUNCH(__half, 4); else PKV_QUANT_LAUNCH(__half, 2);
+    } else {
+        if (E == 4) PKV_QUANT_LAUNCH(float, 4); else PKV_QUANT_LAUNCH(float, 2);
+    }
+#undef PKV_QUANT_LAUNCH
+    return cudaGetLastError();
+}
 
 cudaError_t launch_kv_scatter(const void* src_k, const void* src_v, const int64_t* slots,
                               int64_t num_tokens, void* dst_k, void* dst_v, int64_t row_bytes,

@@ -24,7 +24,7 @@ PKV_F32, PKV_BF16, PKV_F16, PKV_I8 = 0, 1, 2, 3
 _DT = {torch.float32: PKV_F32, torch.bfloat16: PKV_BF16, torch.float16: PKV_F16, torch.int8: PKV_I8}
 
 # every symbol include/pagedkv.h declares
-EXPORTS = ("pkv_error_string", "pkv_kv_cache_write", "pkv_paged_attention_decode",
+EXPORTS = ("pkv_error_string", "pkv_kv_cache_write", "pkv_kv_cache_write_quant", "pkv_paged_attention_decode",
            "pkv_decode_workspace_size", "pkv_decode_plan", "pkv_paged_attention_prefill",
            "pkv_get_device_status")
 
@@ -50,6 +50,8 @@ def load(path: str = _LIB_PATH):
         lib.pkv_error_string.restype = ctypes.c_char_p
         lib.pkv_kv_cache_write.argtypes = [P, P, P, I64, P, P, I, I, I, I64, I, P, P, P, P, P]
         lib.pkv_kv_cache_write.restype = I
+        lib.pkv_kv_cache_write_quant.argtypes = [P, P, I, P, I64, P, P, P, P, I, I, I, I64, P]
+        lib.pkv_kv_cache_write_quant.restype = I
         lib.pkv_paged_attention_decode.argtypes = [P, P, P, P, P, F, P, I, I, I, I, I, I, I64, I, I,
                                                    P, P, P, SZ, I, P]
         lib.pkv_paged_attention_decode.restype = I
@@ -111,6 +113,23 @@ def kv_cache_write(k, v, slot_mapping, k_pages, v_pages, *, k_scale=None, v_scal
                                      _ptr(v_pages), Hkv, D, ps, P, _dtype_code(k_pages), _ptr(k_scale),
                                      _ptr(v_scale), _ptr(k_scale_pages), _ptr(v_scale_pages),
                                      _stream(stream)), "kv_cache_write")
+
+
+def kv_cache_write_quant(k, v, slot_mapping, k_pages, v_pages, k_scale_pages, v_scale_pages, *,
+                         stream=None) -> None:
+    """Quantise new K/V rows ``[T, Hkv, D]`` (bf16/f16/f32) to int8 with one fp16
+    scale per (token, head) and scatter them into the INT8 pools
+    ``[P, ps, Hkv, D]`` and scale pools ``[P, ps, Hkv]`` at ``slot_mapping``."""
+    _cuda(k, v, slot_mapping, k_pages, v_pages, k_scale_pages, v_scale_pages)
+    P, ps, Hkv, D = k_pages.shape
+    if k_pages.dtype != torch.int8 or k_scale_pages.dtype != torch.float16:
+        raise TypeError("INT8 pools and fp16 scale pools expected")
+    if k.shape[1:] != (Hkv, D) or v.shape != k.shape or slot_mapping.dtype != torch.int64:
+        raise ValueError("k/v must be [T, num_kv_heads, head_dim]; slot_mapping int64")
+    _check(load().pkv_kv_cache_write_quant(_ptr(k), _ptr(v), _dtype_code(k), _ptr(slot_mapping), k.shape[0],
+                                           _ptr(k_pages), _ptr(v_pages), _ptr(k_scale_pages),
+                                           _ptr(v_scale_pages), Hkv, D, ps, P, _stream(stream)),
+           "kv_cache_write_quant")
 
 
 def decode_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, page_size, max_pages_per_seq,
