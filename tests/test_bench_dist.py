@@ -1,0 +1,77 @@
+"""bench.py's multi-rank host logic on CPU: world-size-2 gloo ranks, each an
+independent replica; the timed region is the max over ranks and the work
+and units are summed (weak scaling, no data-path collective)."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    import datetime
+
+    import torch.distributed as dist
+
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        assert bench.dist_env() == (rank, world, rank)
+        elapsed, units, work = bench.aggregate(10.0 + 5 * rank, 64.0, 1e9 * (rank + 1))
+        bench.barrier()
+        q.put((rank, elapsed, units, work))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_aggregation_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=10) for _ in range(2))
+    for rank, elapsed, units, work in got:
+        assert elapsed == 15.0                 # max over ranks
+        assert units == 128.0                  # sum over ranks
+        assert work == 3e9
+
+
+def test_single_process_aggregation_is_identity():
+    import bench
+    assert bench.aggregate(3.5, 7, 11) == (3.5, 7, 11)
+
+
+def test_reference_arm_only_rank0_prints(capsys, monkeypatch):
+    import bench
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    bench.run_reference(type("A", (), {"workload": "tiny_decode_f32", "steps": 1, "warmup": 3,
+                                       "ref_seqs": 1, "ref_items": 8})())
+    assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_line_shape(capsys, monkeypatch):
+    import json
+
+    import bench
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    bench.run_reference(type("A", (), {"workload": "tiny_decode_f32", "steps": 2, "warmup": 3,
+                                       "ref_seqs": 2, "ref_items": 8})())
+    line = json.loads(capsys.readouterr().out.strip())
+    assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
