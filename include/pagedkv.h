@@ -166,6 +166,35 @@ int pkv_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
                     int* splits_out, int* split_tokens_out);
 
 /*
+ * Decode attention without any device allocation by the caller.  The pages
+ * have no counterpart: this is a convenience for callers that cannot allocate
+ * device memory on demand (a server that reserved all HBM for its KV-cache
+ * pool at start-up, a plain-C host without a device allocator, a decode loop
+ * that must not risk a synchronising cudaMalloc).  Same arguments and results
+ * as pkv_paged_attention_decode, minus the workspace: the split-KV scratch is
+ * a fixed array of PKV_NOALLOC_SCRATCH_BYTES inside the library, held by
+ * every GPU that loads the library until the process exits.
+ *   - Returns PKV_ERR_WORKSPACE, before launching anything, when these
+ *     arguments need more scratch than that (pkv_decode_workspace_size() >
+ *     PKV_NOALLOC_SCRATCH_BYTES); a smaller num_splits lowers the need.
+ *   - The first call on each device that needs scratch looks up the array's
+ *     device address (cudaGetSymbolAddress); make that first call before any
+ *     stream capture.
+ *   - All calls share the one array: calls that overlap on the GPU (several
+ *     streams or host threads) race on it and must be serialised by the caller.
+ *     Its contents persist between calls; no part of it needs to start zeroed.
+ * The library allocates no device memory on this path either.
+ */
+#define PKV_NOALLOC_SCRATCH_BYTES (48u * 1024u * 1024u)
+int pkv_paged_attention_decode_noalloc(const void* q, const void* k_pages, const void* v_pages,
+                                       const int32_t* block_tables, const int32_t* context_lens,
+                                       float scale, void* out, int num_seqs, int num_q_heads,
+                                       int num_kv_heads, int head_dim, int page_size,
+                                       int max_pages_per_seq, int64_t num_pages, pkv_dtype q_dtype,
+                                       pkv_dtype kv_dtype, const void* k_scales,
+                                       const void* v_scales, int num_splits, pkv_stream_t stream);
+
+/*
  * Chunked prefill attention.  Query rows are packed: rows q_start[b] ..
  * q_start[b+1]-1 are the n_b = q_start[b+1]-q_start[b] new tokens of sequence
  * b, sitting at absolute positions context_lens[b]-n_b .. context_lens[b]-1

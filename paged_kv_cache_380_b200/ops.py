@@ -25,7 +25,8 @@ _DT = {torch.float32: PKV_F32, torch.bfloat16: PKV_BF16, torch.float16: PKV_F16,
 
 # every symbol include/pagedkv.h declares
 EXPORTS = ("pkv_error_string", "pkv_kv_cache_write", "pkv_kv_cache_write_quant", "pkv_paged_attention_decode",
-           "pkv_decode_workspace_size", "pkv_decode_plan", "pkv_paged_attention_prefill",
+           "pkv_decode_workspace_size", "pkv_decode_plan", "pkv_paged_attention_decode_noalloc",
+           "pkv_paged_attention_prefill",
            "pkv_get_device_status")
 
 
@@ -55,6 +56,9 @@ def load(path: str = _LIB_PATH):
         lib.pkv_paged_attention_decode.argtypes = [P, P, P, P, P, F, P, I, I, I, I, I, I, I64, I, I,
                                                    P, P, P, SZ, I, P]
         lib.pkv_paged_attention_decode.restype = I
+        lib.pkv_paged_attention_decode_noalloc.argtypes = [P, P, P, P, P, F, P, I, I, I, I, I, I, I64, I, I,
+                                                           P, P, I, P]
+        lib.pkv_paged_attention_decode_noalloc.restype = I
         lib.pkv_decode_workspace_size.argtypes = [I, I, I, I, I, I, I, I]
         lib.pkv_decode_workspace_size.restype = SZ
         lib.pkv_decode_plan.argtypes = [I, I, I, I, I, I, I, I, ctypes.POINTER(I), ctypes.POINTER(I)]
@@ -174,6 +178,24 @@ def paged_attention_decode(q, k_pages, v_pages, block_tables, context_lens, scal
         _ptr(out), B, Hq, Hkv, D, ps, MP, P, _dtype_code(q), _dtype_code(k_pages), _ptr(k_scales),
         _ptr(v_scales), _ptr(workspace), workspace.numel(), int(num_splits), _stream(stream)),
         "paged_attention_decode")
+    return out
+
+
+def paged_attention_decode_noalloc(q, k_pages, v_pages, block_tables, context_lens, scale, out=None, *,
+                                   k_scales=None, v_scales=None, num_splits=0, stream=None):
+    """Decode attention through the entry point that needs no workspace: the
+    split-KV scratch is a fixed array inside the library (for callers that
+    cannot allocate device memory).  ``out`` must be given by callers that
+    cannot allocate; when omitted it is allocated here with torch."""
+    _cuda(q, k_pages, v_pages, block_tables, context_lens, k_scales, v_scales, out)
+    B, Hq, D = q.shape
+    P, ps, Hkv, _ = k_pages.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _check(load().pkv_paged_attention_decode_noalloc(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_tables), _ptr(context_lens), float(scale), _ptr(out),
+        B, Hq, Hkv, D, ps, block_tables.shape[1], P, _dtype_code(q), _dtype_code(k_pages), _ptr(k_scales),
+        _ptr(v_scales), int(num_splits), _stream(stream)), "paged_attention_decode_noalloc")
     return out
 
 
