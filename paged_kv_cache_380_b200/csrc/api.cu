@@ -20,6 +20,9 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int kChunk = 16;
+#ifndef PKV_SPLIT_MAX_CHUNKS
+#define PKV_SPLIT_MAX_CHUNKS 64   // longest automatic partition: 64 chunks of 16 tokens
+#endif
 
 DeviceStatus* status_ptr() {
     static std::mutex mu;
@@ -75,7 +78,7 @@ Plan plan_decode(int num_seqs, int num_kv_heads, int page_size, int max_pages_pe
     } else {
         const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads;
         const int64_t want = 2LL * sm_count() * 2;   // two waves of two resident CTAs per SM
-        cps = 64;
+        cps = PKV_SPLIT_MAX_CHUNKS;
         while (cps > 16 && units * ((max_chunks + cps - 1) / cps) < want) cps /= 2;
     }
     const int page_chunks = page_size / kChunk > 1 ? page_size / kChunk : 1;

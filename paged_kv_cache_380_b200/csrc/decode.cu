@@ -376,12 +376,19 @@ decode_mma_kernel(const DecodeParams p) {
     }
 }
 
-// Merge of the split-KV partials of one (sequence, query head) per warp.
+// Merge of the split-KV partials: one CTA per (sequence, query head), its 8
+// warps striding over the partitions (each warp reads whole 512-byte partial
+// rows, four in flight), then a shared-memory sum across the warps.  Weights
+// 2^(lse_p - max) against the global max of the partitions' log2-sum-exps.
+constexpr int kCombineWarps = 8;
+
 template <typename QT, int HD>
-__global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kCombineWarps * 32) decode_combine_kernel(const DecodeParams p) {
+    __shared__ float sm_max[kCombineWarps];
+    __shared__ float sm_w[kCombineWarps];
+    __shared__ float sm_acc[kCombineWarps][HD];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int gw = blockIdx.x * 4 + warp;
-    if (gw >= p.num_seqs * p.num_q_heads) return;
+    const int gw = blockIdx.x;                                   // b * Hq + h
     const int b = gw / p.num_q_heads;
     const int ctx = __ldg(p.context_lens + b);
     if (ctx <= 0 || ctx > p.max_pages_per_seq * p.page_size) return;
@@ -390,31 +397,44 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
     const float* lse = p.lse_part + static_cast<size_t>(gw) * p.max_splits;
     const float* op = p.o_part + static_cast<size_t>(gw) * p.max_splits * HD;
     float M = -INFINITY;
-    for (int s = lane; s < ns; s += 32) M = fmaxf(M, lse[s]);
+    for (int s = threadIdx.x; s < ns; s += kCombineWarps * 32) M = fmaxf(M, lse[s]);
 #pragma unroll
     for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
+    if (lane == 0) sm_max[warp] = M;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < kCombineWarps; ++w) M = fmaxf(M, sm_max[w]);
     constexpr int E = HD / 32;
     float acc[E];
 #pragma unroll
     for (int j = 0; j < E; ++j) acc[j] = 0.f;
-    float W = 0.f;
+    float wsum = 0.f;
 #pragma unroll 4
-    for (int s = 0; s < ns; ++s) {
+    for (int s = warp; s < ns; s += kCombineWarps) {
         const float w = ptx::ex2(lse[s] - M);
-        W += w;
+        wsum += w;
         const float* src = op + static_cast<size_t>(s) * HD + lane * E;
         if constexpr (E == 4) {
             const float4 v = *reinterpret_cast<const float4*>(src);
             acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
         } else {
-#pragma unroll
-            for (int j = 0; j < E; ++j) acc[j] += w * src[j];
+            const float2 v = *reinterpret_cast<const float2*>(src);
+            acc[0] += w * v.x; acc[1] += w * v.y;
         }
     }
-    QT* out = static_cast<QT*>(p.out) + static_cast<size_t>(gw) * HD + lane * E;
-    const float inv = 1.f / W;
 #pragma unroll
-    for (int j = 0; j < E; ++j) out[j] = from_float<QT>(acc[j] * inv);
+    for (int j = 0; j < E; ++j) sm_acc[warp][lane * E + j] = acc[j];
+    if (lane == 0) sm_w[warp] = wsum;
+    __syncthreads();
+    if (threadIdx.x < HD) {
+        float a = 0.f, wt = 0.f;
+#pragma unroll
+        for (int w = 0; w < kCombineWarps; ++w) {
+            a += sm_acc[w][threadIdx.x];
+            wt += sm_w[w];
+        }
+        static_cast<QT*>(p.out)[static_cast<size_t>(gw) * HD + threadIdx.x] = from_float<QT>(a / wt);
+    }
 }
 
 // fp32 pages and queries (small problems; CUDA-core path with exact-ish fp32
@@ -467,8 +487,14 @@ __global__ void __launch_bounds__(128) decode_f32_kernel(const DecodeParams p) {
     }
 }
 
-constexpr int kWarps = 4;
-constexpr int kStages = 3;
+#ifndef PKV_DECODE_WARPS
+#define PKV_DECODE_WARPS 4
+#endif
+#ifndef PKV_DECODE_STAGES
+#define PKV_DECODE_STAGES 3
+#endif
+constexpr int kWarps = PKV_DECODE_WARPS;    // warps per CTA, each with its own cp.async ring
+constexpr int kStages = PKV_DECODE_STAGES;  // ring depth (16-token chunks)
 
 template <typename QT, typename KVT, int HD, int NT>
 cudaError_t run_mma(const DecodeParams& p, cudaStream_t stream) {
@@ -480,8 +506,7 @@ cudaError_t run_mma(const DecodeParams& p, cudaStream_t stream) {
     kern<<<grid, kWarps * 32, Cfg::kSmem, stream>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || p.max_splits == 1) return e;
-    const int warps = p.num_seqs * p.num_q_heads;
-    decode_combine_kernel<QT, HD><<<ceil_div(warps, 4), 128, 0, stream>>>(p);
+    decode_combine_kernel<QT, HD><<<p.num_seqs * p.num_q_heads, kCombineWarps * 32, 0, stream>>>(p);
     return cudaGetLastError();
 }
 

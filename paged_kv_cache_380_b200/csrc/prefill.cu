@@ -19,9 +19,12 @@
 //    bf16 -> fp32 in TMEM, triple-buffered) and O += P_j V_j with P read from
 //    TMEM (the TS form) and V as an MN-major operand; tcgen05.commit signals
 //    S ready, the K stage free, O updated and the V stage free.
-//  * warps 2-5 = softmax: one TMEM lane (query row) per thread; tcgen05.ld of
-//    the S row, masking, row max, exp2, row sum, P packed to bf16 pairs and
-//    tcgen05.st back over the S columns.  The accumulator is rescaled only
+//  * warps 2-9 = softmax: one TMEM lane (query row) per thread, two warps per
+//    row quarter taking 64 columns each (row max and row sum exchanged in
+//    shared memory); tcgen05.ld of the S half-row, masking, max, 2^(s*scale -
+//    m) with the scale folded into one FFMA (one exponential in four on the
+//    FMA pipe as a polynomial, the rest on the SFU), row sum, P packed to bf16
+//    pairs and tcgen05.st back over the S columns.  The accumulator is rescaled only
 //    when a row's running max grows by more than 2^8 (P <= 256 otherwise),
 //    which keeps O's TMEM round trip off most tiles; the final division by
 //    the row sum makes any consistent reference max exact.
@@ -44,18 +47,46 @@ namespace {
 
 constexpr int BM = 128, BN = 128, HD = 128;
 constexpr int KST = 3, VST = 2, NSB = 3;        // K stages, V stages, S/P TMEM buffers
-constexpr int kThreads = 192;
+constexpr int kProducerWarps = 3;               // TMA issue is split over three warps
+constexpr int kMmaWarp = kProducerWarps;
+constexpr int kSoftmaxWarp0 = kMmaWarp + 1;
+constexpr int kSoftmaxWarps = 8;                // two warps per TMEM lane quarter, 64 columns each
+constexpr int kThreads = (kSoftmaxWarp0 + kSoftmaxWarps) * 32;   // 12 warps = 3 warpgroups
 constexpr int kAtom = BN * 128;                 // one 64-column SW128 half of a 128-row tile
 constexpr int kTile = 2 * kAtom;                // 32 KB
 constexpr int kSmemQ = 0;
 constexpr int kSmemK = kSmemQ + kTile;
 constexpr int kSmemV = kSmemK + KST * kTile;
-constexpr int kSmemBar = kSmemV + VST * kTile;
+constexpr int kSmemRed = kSmemV + VST * kTile;   // row-max / row-sum exchange between warp pairs
+constexpr int kRedBytes = (2 * 2 * BM + 2 * BM) * 4;
+constexpr int kSmemBar = kSmemRed + kRedBytes;
 constexpr int kNumBars = 1 + 2 * KST + 2 * VST + 3 * NSB + 1;
 constexpr int kSmemBytes = kSmemBar + kNumBars * 8 + 16 + 1024;   // + TMEM addr, abort flag, alignment
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kOCol = NSB * 128;           // O accumulator columns 384..511
 constexpr float kRescaleThreshold = 8.0f;       // log2 units: rescale when the max grows by > 2^8
+#ifndef PKV_PREFILL_POLY_EVERY
+#define PKV_PREFILL_POLY_EVERY 0                 // 1 in N exponentials on the FMA pipe (0 = none)
+#endif
+constexpr int kPolyEvery = PKV_PREFILL_POLY_EVERY;
+
+// 2^x on the FMA/ALU pipes, for softmax arguments x <= 8: Cody-Waite split
+// x = n + f with n = round(x) (the 1.5 * 2^23 shifter), f in [-0.5, 0.5];
+// 2^f from a degree-3 polynomial fitted here for least relative error on
+// [-0.5, 0.5] (iteratively reweighted least squares, max relative error
+// 7.5e-5, below the bf16 rounding P gets anyway); 2^n added into the
+// exponent field.  Arguments below -126 are clamped (result ~1e-38 instead of 0).
+__device__ __forceinline__ float exp2_poly(float x) {
+    x = fmaxf(x, -126.0f);
+    const float t = x + 12582912.0f;
+    const float f = x - (t - 12582912.0f);
+    const float q = fmaf(fmaf(fmaf(0.055166300f, f, 0.24261182f), f, 0.69326228f), f, 0.99992806f);
+    return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");
+}
 
 // sm_100 shared-memory matrix descriptor: start, leading and stride byte
 // offsets (>> 4), version 1, SWIZZLE_128B layout.
@@ -125,25 +156,53 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
     const int max_key = p.causal ? ctx - n + last_row : ctx - 1;
     const int n_tiles = max_key / BN + 1;
     const int min_lim = p.causal ? ctx - n + r0 : ctx - 1;      // every row of the tile sees keys <= this
+    // Tiles every row sees in full are visited in a rotated order that differs
+    // between the CTAs reading the same pages (query heads of one KV head, and
+    // sequences sharing a prefix), so concurrent CTAs do not all fetch the same
+    // lines at once; masked (diagonal / last) tiles follow in order.
+#ifndef PKV_PREFILL_ROTATE
+#define PKV_PREFILL_ROTATE 1
+#endif
+    const int n_full = min((min_lim + 1) / BN, n_tiles);
+    const int rot = (PKV_PREFILL_ROTATE && n_full > 1) ? (h * 3 + b * 5) % n_full : 0;
+    auto tile_of = [&](int j) { return j < n_full ? (j + rot) % n_full : j; };
 
     const Bars bars{sbase + kSmemBar};
+    // Page indices, 4 tiles (32 groups of 16 keys) per batch: lane i of batch k holds the
+    // physical page of group i%8 of tile 4k + i/8 (loaded by the producer warp only).
+    const int32_t* bt = p.block_tables + static_cast<size_t>(b) * p.max_pages_per_seq;
+    auto load_pages = [&](int k) -> int {
+        const int key0 = tile_of(4 * k + (lane >> 3)) * BN + 16 * (lane & 7);
+        return key0 < ctx ? __ldg(bt + key0 / ps) : -1;
+    };
+    int pg_cur = 0, pg_next = 0;
+    if (warp < kProducerWarps) {
+        pg_cur = load_pages(0);
+        pg_next = load_pages(1);
+    }
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kSmemBar + kNumBars * 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSmemBar + kNumBars * 8 + 8);
 
     if (threadIdx.x == 0) {
         ptx::mbar_init(bars.q_full(), 1);
-        for (int i = 0; i < KST; ++i) { ptx::mbar_init(bars.k_full(i), 1); ptx::mbar_init(bars.k_empty(i), 1); }
-        for (int i = 0; i < VST; ++i) { ptx::mbar_init(bars.v_full(i), 1); ptx::mbar_init(bars.v_empty(i), 1); }
+        for (int i = 0; i < KST; ++i) {
+            ptx::mbar_init(bars.k_full(i), kProducerWarps);
+            ptx::mbar_init(bars.k_empty(i), 1);
+        }
+        for (int i = 0; i < VST; ++i) {
+            ptx::mbar_init(bars.v_full(i), kProducerWarps);
+            ptx::mbar_init(bars.v_empty(i), 1);
+        }
         for (int i = 0; i < NSB; ++i) {
             ptx::mbar_init(bars.s_full(i), 1);
-            ptx::mbar_init(bars.p_full(i), 128);
+            ptx::mbar_init(bars.p_full(i), kSoftmaxWarps * 32);
             ptx::mbar_init(bars.pv_done(i), 1);
         }
         ptx::mbar_init(bars.mma_done(), 1);
         *abort_flag = 0;
         ptx::fence_mbarrier_init();
     }
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
         ptx::tmem_relinquish();
     }
@@ -152,10 +211,15 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
-        // ------------------------------ TMA producer ------------------------------
-        const int32_t* bt = p.block_tables + static_cast<size_t>(b) * p.max_pages_per_seq;
-        if (lane == 0) {
+    if (warp < kProducerWarps) {
+        // ------------------------------ TMA producers ------------------------------
+        // A tile is 8 page groups x 2 column halves = 16 boxes per tensor; producer
+        // warp w issues the boxes of groups w, w+3, w+6 (one box per lane), because a
+        // single issuing warp cannot keep enough 2 KB boxes in flight.  K runs up to KST
+        // tiles ahead; V is issued one tile behind K so that waiting for a free V
+        // stage never delays the next K tile.  Page indices come from register
+        // batches loaded four tiles ahead (pg_cur / pg_next).
+        if (warp == 0 && lane == 0) {
             ptx::prefetch_tmap(&tm_q);
             ptx::prefetch_tmap(&tm_k);
             ptx::prefetch_tmap(&tm_v);
@@ -163,41 +227,52 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
             ptx::tma_load_3d(sbase + kSmemQ, &tm_q, bars.q_full(), 0, h, q0 + r0);
             ptx::tma_load_3d(sbase + kSmemQ + kAtom, &tm_q, bars.q_full(), 64, h, q0 + r0);
         }
-        bool ok = true;
-        for (int t = 0; t < n_tiles && ok; ++t) {
-            // lane g < 8 resolves the page of 16-key group g of this tile
-            const int key0 = t * BN + 16 * (lane & 7);
+        const int my_group = warp + kProducerWarps * (lane >> 1);   // lane pair -> one page group
+        const int my_half = lane & 1;
+        const bool my_lane = my_group < 8;
+        // TMA row (slot) of my page group in tile t, or -1 (past the context / bad page)
+        auto row_of = [&](int t, int pg_word) -> int {
+            const int page = __shfl_sync(0xffffffffu, pg_word, (t & 3) * 8 + (my_group & 7));
+            const int key0 = tile_of(t) * BN + 16 * my_group;
+            if (!my_lane || key0 >= ctx) return -1;
+            if (page < 0 || page >= p.num_pages) {
+                if (my_half == 0) record_error(p.status, PKV_ERR_DEVICE_RANGE, page);
+                return -1;
+            }
+            return page * ps + key0 % ps;
+        };
+        auto issue = [&](bool is_k, int t, int row) -> bool {
+            const int nst = is_k ? KST : VST, st = t % nst;
+            const unsigned nbox = __popc(__ballot_sync(0xffffffffu, row >= 0));
+            bool ok = true;
+            if (t >= nst)
+                ok = wait_bar(is_k ? bars.k_empty(st) : bars.v_empty(st), ((t / nst) - 1) & 1, abort_flag, p.status);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok) return false;
+            const uint32_t bar = is_k ? bars.k_full(st) : bars.v_full(st);
+            if (lane == 0) ptx::mbar_arrive_expect_tx(bar, nbox * 16 * 128);
+            __syncwarp();
+            if (row >= 0) {
+                const uint32_t dst = sbase + (is_k ? kSmemK : kSmemV) + st * kTile + my_half * kAtom + my_group * 2048;
+                ptx::tma_load_3d(dst, is_k ? &tm_k : &tm_v, bar, 64 * my_half, kvh, row);
+            }
+            return true;
+        };
+        int row_prev = -1;
+        for (int t = 0; t <= n_tiles; ++t) {
             int row = -1;
-            if (lane < 8 && key0 < ctx) {
-                const int page = __ldg(bt + key0 / ps);
-                if (page >= 0 && page < p.num_pages) row = page * ps + key0 % ps;
-                else record_error(p.status, PKV_ERR_DEVICE_RANGE, page);
+            if (t < n_tiles) {
+                if (t > 0 && (t & 3) == 0) {
+                    pg_cur = pg_next;
+                    pg_next = load_pages(t / 4 + 1);
+                }
+                row = row_of(t, pg_cur);
+                if (!issue(true, t, row)) break;
             }
-            const unsigned valid = __ballot_sync(0xffffffffu, row >= 0) & 0xffu;
-            const uint32_t bytes = __popc(valid) * 16 * 128 * 2;
-            const int ks = t % KST, vs = t % VST;
-            if (t >= KST) ok = wait_bar(bars.k_empty(ks), ((t / KST) - 1) & 1, abort_flag, p.status);
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!ok) break;
-            if (lane == 0) ptx::mbar_arrive_expect_tx(bars.k_full(ks), bytes);
-            __syncwarp();
-            if (row >= 0) {
-                const uint32_t dst = sbase + kSmemK + ks * kTile + (lane & 7) * 2048;
-                ptx::tma_load_3d(dst, &tm_k, bars.k_full(ks), 0, kvh, row);
-                ptx::tma_load_3d(dst + kAtom, &tm_k, bars.k_full(ks), 64, kvh, row);
-            }
-            if (t >= VST) ok = wait_bar(bars.v_empty(vs), ((t / VST) - 1) & 1, abort_flag, p.status);
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!ok) break;
-            if (lane == 0) ptx::mbar_arrive_expect_tx(bars.v_full(vs), bytes);
-            __syncwarp();
-            if (row >= 0) {
-                const uint32_t dst = sbase + kSmemV + vs * kTile + (lane & 7) * 2048;
-                ptx::tma_load_3d(dst, &tm_v, bars.v_full(vs), 0, kvh, row);
-                ptx::tma_load_3d(dst + kAtom, &tm_v, bars.v_full(vs), 64, kvh, row);
-            }
+            if (t >= 1 && !issue(false, t - 1, row_prev)) break;
+            row_prev = row;
         }
-    } else if (warp == 1) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------ MMA issuer ------------------------------
         if (lane == 0) {
             constexpr uint32_t id_s = idesc_f16<T>(BM, BN, 0);
@@ -241,9 +316,15 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
         }
     } else {
         // ------------------------------ softmax + epilogue ------------------------------
-        const int quarter = warp & 3;
+        // Warp w reaches TMEM lanes 32*(w%4)..+31 (its quarter of the rows); the two
+        // warps of a quarter split the 128 columns of S (and of O) into halves and
+        // exchange row maxima (and finally row sums) through shared memory.
+        const int quarter = warp & 3, hf = (warp - kSoftmaxWarp0) >> 2;
         const int row = quarter * 32 + lane;                        // TMEM lane == tile row
         const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        const int c0 = hf * 64;                                     // this warp's S / O columns
+        float* red = reinterpret_cast<float*>(smem + kSmemRed);     // [2 bufs][2 halves][BM]
+        float* lsum = red + 2 * 2 * BM;                             // [2 halves][BM]
         const int lim = min(p.causal ? ctx - n + r0 + row : ctx - 1, ctx - 1);
         const float sl2 = p.scale_log2;
         float m_ref = -INFINITY, l = 0.f;
@@ -253,79 +334,85 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
             ok = wait_bar(bars.s_full(bj), (j / NSB) & 1, abort_flag, p.status);
             if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
             ptx::tc_fence_after();
-            float x[BN];
-#pragma unroll
-            for (int c4 = 0; c4 < BN / 32; ++c4) {
-                uint32_t r[32];
-                ptx::tmem_ld32(trow + bj * 128 + c4 * 32, r);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) x[c4 * 32 + i] = __uint_as_float(r[i]);
+            uint32_t r[64];
+            {
+                uint32_t (&r0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[0]);
+                uint32_t (&r1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[32]);
+                ptx::tmem_ld32(trow + bj * 128 + c0, r0);
+                ptx::tmem_ld32(trow + bj * 128 + c0 + 32, r1);
             }
             ptx::tc_wait_ld();
-            const bool need_mask = j * BN + BN - 1 > min_lim;
-            float mt = -INFINITY;
+            float x[64];
 #pragma unroll
-            for (int c = 0; c < BN; ++c) {
-                float v = x[c] * sl2;
-                if (need_mask && j * BN + c > lim) v = -INFINITY;
-                x[c] = v;
-                mt = fmaxf(mt, v);
+            for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(r[c]);
+            const int jt = tile_of(j);
+            if (jt * BN + BN - 1 > min_lim) {                       // diagonal / last tile: mask
+#pragma unroll
+                for (int c = 0; c < 64; ++c)
+                    if (jt * BN + c0 + c > lim) x[c] = -INFINITY;
             }
+            float mh = x[0];
+#pragma unroll
+            for (int c = 1; c < 64; ++c) mh = fmaxf(mh, x[c]);
+            float* rb = red + (j & 1) * 2 * BM;
+            rb[hf * BM + row] = mh;
+            named_bar_sync(1 + quarter, 64);
+            const float mt = fmaxf(mh, rb[(1 - hf) * BM + row]) * sl2;   // finite: key 0 is visible
             if (j == 0) {
-                m_ref = mt;                                         // finite: key 0 is always visible
-            } else {
-                const bool want = mt > m_ref + kRescaleThreshold;
-                if (__any_sync(0xffffffffu, want)) {
-                    const float m_new = fmaxf(m_ref, mt);
-                    const float corr = ptx::ex2(m_ref - m_new);
-                    l *= corr;
-                    m_ref = m_new;
-                    const int pj = j - 1;
-                    ok = wait_bar(bars.pv_done(pj % NSB), (pj / NSB) & 1, abort_flag, p.status);
-                    if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
-                    ptx::tc_fence_after();
+                m_ref = mt;
+            } else if (__any_sync(0xffffffffu, mt > m_ref + kRescaleThreshold)) {
+                const float m_new = fmaxf(m_ref, mt);
+                const float corr = ptx::ex2(m_ref - m_new);
+                l *= corr;
+                m_ref = m_new;
+                const int pj = j - 1;
+                ok = wait_bar(bars.pv_done(pj % NSB), (pj / NSB) & 1, abort_flag, p.status);
+                if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+                ptx::tc_fence_after();
 #pragma unroll
-                    for (int c4 = 0; c4 < HD / 32; ++c4) {
-                        uint32_t r[32];
-                        ptx::tmem_ld32(trow + kOCol + c4 * 32, r);
-                        ptx::tc_wait_ld();
-                        uint32_t w0[16], w1[16];
+                for (int c32 = 0; c32 < 2; ++c32) {
+                    uint32_t o[32];
+                    ptx::tmem_ld32(trow + kOCol + c0 + c32 * 32, o);
+                    ptx::tc_wait_ld();
+                    uint32_t w0[16], w1[16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            w0[i] = __float_as_uint(__uint_as_float(r[i]) * corr);
-                            w1[i] = __float_as_uint(__uint_as_float(r[16 + i]) * corr);
-                        }
-                        ptx::tmem_st16(trow + kOCol + c4 * 32, w0);
-                        ptx::tmem_st16(trow + kOCol + c4 * 32 + 16, w1);
+                    for (int i = 0; i < 16; ++i) {
+                        w0[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
+                        w1[i] = __float_as_uint(__uint_as_float(o[16 + i]) * corr);
                     }
-                    ptx::tc_wait_st();
+                    ptx::tmem_st16(trow + kOCol + c0 + c32 * 32, w0);
+                    ptx::tmem_st16(trow + kOCol + c0 + c32 * 32 + 16, w1);
                 }
+                ptx::tc_wait_st();
             }
+            const float neg = -m_ref;
             float rs = 0.f;
 #pragma unroll
-            for (int c16 = 0; c16 < BN / 32; ++c16) {
+            for (int c16 = 0; c16 < 2; ++c16) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const float a = ptx::ex2(x[c16 * 32 + 2 * i] - m_ref);
-                    const float bb = ptx::ex2(x[c16 * 32 + 2 * i + 1] - m_ref);
+                    const int c = c16 * 32 + 2 * i;
+                    const float ya = fmaf(x[c], sl2, neg), yb = fmaf(x[c + 1], sl2, neg);
+                    const float a = (kPolyEvery && (c % kPolyEvery) == kPolyEvery - 1) ? exp2_poly(ya) : ptx::ex2(ya);
+                    const float bb = (kPolyEvery && ((c + 1) % kPolyEvery) == kPolyEvery - 1) ? exp2_poly(yb) : ptx::ex2(yb);
                     rs += a + bb;
                     pk[i] = pack2<T>(a, bb);
                 }
-                ptx::tmem_st16(trow + bj * 128 + c16 * 16, pk);
+                ptx::tmem_st16(trow + bj * 128 + hf * 32 + c16 * 16, pk);
             }
             l += rs;
             ptx::tc_wait_st();
-            if (j == n_tiles - 1 && ctx < (j + 1) * BN) {
+            if (ctx < (jt + 1) * BN) {
                 // V rows past the context (tail of the last page, or never loaded) must be
                 // finite zeros: P is 0 there but 0 * NaN would poison O.
                 const int vs = j % VST;
                 ok = wait_bar(bars.v_full(vs), (j / VST) & 1, abort_flag, p.status);
                 if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
-                const int first = ctx - j * BN;                     // first invalid row of the tile
+                const int first = ctx - jt * BN;                    // first invalid row of the tile
                 uint4* vt = reinterpret_cast<uint4*>(smem + kSmemV + vs * kTile);
-                const int tid = threadIdx.x - 64;
-                for (int idx = tid; idx < 2 * (BN - first) * 8; idx += 128) {
+                const int tid = threadIdx.x - kSoftmaxWarp0 * 32;
+                for (int idx = tid; idx < 2 * (BN - first) * 8; idx += kSoftmaxWarps * 32) {
                     const int half = idx / ((BN - first) * 8), rem = idx % ((BN - first) * 8);
                     vt[(half * kAtom + (first + rem / 8) * 128) / 16 + rem % 8] = make_uint4(0, 0, 0, 0);
                 }
@@ -334,27 +421,29 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
             ptx::tc_fence_before();
             ptx::mbar_arrive(bars.p_full(bj));
         }
-        // epilogue: O / l -> out
+        // epilogue: O / l -> out (each warp writes its 64 output columns)
         if (ok) {
             const int pj = n_tiles - 1;
             ok = wait_bar(bars.pv_done(pj % NSB), (pj / NSB) & 1, abort_flag, p.status);
         }
+        lsum[hf * BM + row] = l;
+        named_bar_sync(1 + quarter, 64);
         if (__all_sync(0xffffffffu, ok)) {
             ptx::tc_fence_after();
-            const float inv = 1.f / l;
+            const float inv = 1.f / (l + lsum[(1 - hf) * BM + row]);
             const bool store = r0 + row < n;
-            T* out = static_cast<T*>(p.out) + (static_cast<size_t>(q0 + r0 + row) * Hq + h) * HD;
+            T* out = static_cast<T*>(p.out) + (static_cast<size_t>(q0 + r0 + row) * Hq + h) * HD + c0;
 #pragma unroll
-            for (int c4 = 0; c4 < HD / 32; ++c4) {
-                uint32_t r[32];
-                ptx::tmem_ld32(trow + kOCol + c4 * 32, r);
+            for (int c32 = 0; c32 < 2; ++c32) {
+                uint32_t o[32];
+                ptx::tmem_ld32(trow + kOCol + c0 + c32 * 32, o);
                 ptx::tc_wait_ld();
                 uint32_t w[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
-                    w[i] = pack2<T>(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+                    w[i] = pack2<T>(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
                 if (store) {
-                    uint4* dst = reinterpret_cast<uint4*>(out + c4 * 32);
+                    uint4* dst = reinterpret_cast<uint4*>(out + c32 * 32);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
                 }
@@ -368,7 +457,7 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
         // let in-flight TMA writes land before the shared memory is handed to another CTA
         for (int t = 0; t < KST; ++t) ptx::mbar_wait(bars.k_full(t), 0, kSpinLimit >> 4);
     }
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, kTmemCols);
     }
