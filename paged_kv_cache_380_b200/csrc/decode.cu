@@ -48,14 +48,15 @@ namespace {
 constexpr int kChunk = 16;            // tokens per pipeline stage of one warp
 constexpr unsigned kFull = 0xffffffffu;
 
-// int8 code pair (bytes a, b of w) -> two MMA-type values, exact: the byte,
-// offset by 128, becomes the low mantissa bits of 2^23 (fp32), then the offset
-// is subtracted; |code| <= 128 is exact in bf16 and fp16.
-template <typename QT>
+// int8 code pair (bytes a, b of w, each offset by 128 through w ^ 0x80808080)
+// -> fp16x2, exact: the offset byte u becomes the low mantissa byte of the fp16
+// number 1024 + u (exponent pattern 0x64), then 1152 = 1024 + 128 is subtracted
+// from both halves at once; |code| <= 128 is exact in fp16.
 __device__ __forceinline__ uint32_t s8pair(uint32_t w_biased, uint32_t sel_a, uint32_t sel_b) {
-    const float fa = __int_as_float(__byte_perm(w_biased, 0x4B000000u, 0x7540u | sel_a)) - 8388736.0f;
-    const float fb = __int_as_float(__byte_perm(w_biased, 0x4B000000u, 0x7540u | sel_b)) - 8388736.0f;
-    return pack2<QT>(fa, fb);
+    const uint32_t h = __byte_perm(w_biased, 0x64646464u, sel_a | 0x40u | (sel_b << 8) | 0x4000u);
+    __half2 x = *reinterpret_cast<const __half2*>(&h);
+    x = __hsub2(x, __half2half2(__ushort_as_half(0x6480)));   // 0x6480 = 1152.0
+    return *reinterpret_cast<uint32_t*>(&x);
 }
 
 template <typename QT>
@@ -87,6 +88,8 @@ template <typename QT, typename KVT, int HD, int NT, int WARPS, int STAGES>
 __global__ void __launch_bounds__(WARPS * 32)
 decode_mma_kernel(const DecodeParams p) {
     using Cfg = DecodeCfg<QT, KVT, HD, NT, WARPS, STAGES>;
+    // INT8 pages run the MMAs in fp16 (codes widen to fp16 in two instructions per pair)
+    using MT = typename std::conditional<Cfg::kInt8, __half, QT>::type;
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
@@ -127,6 +130,39 @@ decode_mma_kernel(const DecodeParams p) {
                 qf[nt][kk][0] = n < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + d0)) : 0u;
                 qf[nt][kk][1] = n < G ? __ldg(reinterpret_cast<const uint32_t*>(qrow + d1)) : 0u;
             }
+        }
+    }
+    // INT8 pages: q goes to fp16 for the MMA.  Each head is first scaled by a power
+    // of two (exact) so that its largest |q| stays below 2^15; the inverse factor
+    // multiplies that head's scores.  qinv[nt][h] is the factor of head 2c + h.
+    float qinv[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) qinv[nt][0] = qinv[nt][1] = 1.f;
+    if constexpr (Cfg::kInt8) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            float mq = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < Cfg::kDT; ++kk)
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const float2 v = unpack2<QT>(qf[nt][kk][i]);
+                    mq = fmaxf(mq, fmaxf(fabsf(v.x), fabsf(v.y)));
+                }
+            mq = fmaxf(mq, __shfl_xor_sync(kFull, mq, 1));
+            mq = fmaxf(mq, __shfl_xor_sync(kFull, mq, 2));
+            const int e = ((__float_as_int(mq) >> 23) & 0xff) - 127;      // floor(log2(max |q|))
+            const float f = e >= 15 ? __int_as_float((127 + 14 - e) << 23) : 1.f;
+#pragma unroll
+            for (int kk = 0; kk < Cfg::kDT; ++kk)
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const float2 v = unpack2<QT>(qf[nt][kk][i]);
+                    qf[nt][kk][i] = pack2<__half>(v.x * f, v.y * f);
+                }
+            const float inv = 1.f / f;                                    // exact: a power of two
+            qinv[nt][0] = __shfl_sync(kFull, inv, (2 * c) * 4);
+            qinv[nt][1] = __shfl_sync(kFull, inv, (2 * c + 1) * 4);
         }
     }
 
@@ -218,10 +254,10 @@ decode_mma_kernel(const DecodeParams p) {
                     // w0: rows 0-7 unit U, w1: rows 8-15 unit U, w2/w3: unit U+1
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
-                        mma16816<QT>(s[nt], s8pair<QT>(w0, 0, 1), s8pair<QT>(w1, 0, 1), s8pair<QT>(w0, 2, 3),
-                                     s8pair<QT>(w1, 2, 3), qf[nt][U][0], qf[nt][U][1]);
-                        mma16816<QT>(s[nt], s8pair<QT>(w2, 0, 1), s8pair<QT>(w3, 0, 1), s8pair<QT>(w2, 2, 3),
-                                     s8pair<QT>(w3, 2, 3), qf[nt][U + 1][0], qf[nt][U + 1][1]);
+                        mma16816<MT>(s[nt], s8pair(w0, 0, 1), s8pair(w1, 0, 1), s8pair(w0, 2, 3),
+                                     s8pair(w1, 2, 3), qf[nt][U][0], qf[nt][U][1]);
+                        mma16816<MT>(s[nt], s8pair(w2, 0, 1), s8pair(w3, 0, 1), s8pair(w2, 2, 3),
+                                     s8pair(w3, 2, 3), qf[nt][U + 1][0], qf[nt][U + 1][1]);
                     }
                 }
             }
@@ -248,10 +284,10 @@ decode_mma_kernel(const DecodeParams p) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             float x[4];
-            x[0] = va ? s[nt][0] * (p.scale_log2 * ks_a) : -INFINITY;
-            x[1] = va ? s[nt][1] * (p.scale_log2 * ks_a) : -INFINITY;
-            x[2] = vb ? s[nt][2] * (p.scale_log2 * ks_b) : -INFINITY;
-            x[3] = vb ? s[nt][3] * (p.scale_log2 * ks_b) : -INFINITY;
+            x[0] = va ? s[nt][0] * (p.scale_log2 * ks_a * qinv[nt][0]) : -INFINITY;
+            x[1] = va ? s[nt][1] * (p.scale_log2 * ks_a * qinv[nt][1]) : -INFINITY;
+            x[2] = vb ? s[nt][2] * (p.scale_log2 * ks_b * qinv[nt][0]) : -INFINITY;
+            x[3] = vb ? s[nt][3] * (p.scale_log2 * ks_b * qinv[nt][1]) : -INFINITY;
             float pr[4];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -272,8 +308,8 @@ decode_mma_kernel(const DecodeParams p) {
                 }
             }
             // P^T fragments (B operand of O^T += V^T . P^T) via 8x8 transposes
-            pb[nt][0] = ptx::movmatrix_trans(pack2<QT>(pr[0] * vs_a, pr[1] * vs_a));
-            pb[nt][1] = ptx::movmatrix_trans(pack2<QT>(pr[2] * vs_b, pr[3] * vs_b));
+            pb[nt][0] = ptx::movmatrix_trans(pack2<MT>(pr[0] * vs_a, pr[1] * vs_a));
+            pb[nt][1] = ptx::movmatrix_trans(pack2<MT>(pr[2] * vs_b, pr[3] * vs_b));
         }
 
         // ---- O^T += V^T . P^T ----
@@ -297,10 +333,10 @@ decode_mma_kernel(const DecodeParams p) {
                 w0 ^= 0x80808080u; w1 ^= 0x80808080u; w2 ^= 0x80808080u; w3 ^= 0x80808080u;
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    mma16816<QT>(o[nt][U], s8pair<QT>(w0, 0, 2), s8pair<QT>(w0, 1, 3), s8pair<QT>(w1, 0, 2),
-                                 s8pair<QT>(w1, 1, 3), pb[nt][0], pb[nt][1]);
-                    mma16816<QT>(o[nt][U + 1], s8pair<QT>(w2, 0, 2), s8pair<QT>(w2, 1, 3), s8pair<QT>(w3, 0, 2),
-                                 s8pair<QT>(w3, 1, 3), pb[nt][0], pb[nt][1]);
+                    mma16816<MT>(o[nt][U], s8pair(w0, 0, 2), s8pair(w0, 1, 3), s8pair(w1, 0, 2),
+                                 s8pair(w1, 1, 3), pb[nt][0], pb[nt][1]);
+                    mma16816<MT>(o[nt][U + 1], s8pair(w2, 0, 2), s8pair(w2, 1, 3), s8pair(w3, 0, 2),
+                                 s8pair(w3, 1, 3), pb[nt][0], pb[nt][1]);
                 }
             }
         }

@@ -58,6 +58,15 @@ template <> __device__ __forceinline__ uint32_t pack2<__half>(float a, float b) 
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Unpack a 32-bit pair of 16-bit values (low half first) to two floats.
+template <typename T> __device__ __forceinline__ float2 unpack2(uint32_t v);
+template <> __device__ __forceinline__ float2 unpack2<__nv_bfloat16>(uint32_t v) {
+    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+}
+template <> __device__ __forceinline__ float2 unpack2<__half>(uint32_t v) {
+    return __half22float2(*reinterpret_cast<const __half2*>(&v));
+}
+
 __host__ __device__ constexpr inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 }  // namespace pkv

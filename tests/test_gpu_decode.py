@@ -144,3 +144,14 @@ def test_out_of_range_page_is_recorded_not_faulted():
     want = oracle.decode(c.q, "bf16", c.k_pages, c.v_pages, "bf16", c.block_tables, c.context_lens, c.scale)
     assert_close(f64(out)[0], want[0], 2e-2, "unaffected sequence")
     assert_status_ok()
+
+
+def test_int8_pages_large_queries():
+    """Queries far beyond the fp16 range (bf16 allows them): the INT8 path scales each
+    head by a power of two before its fp16 MMA and folds the factor back exactly."""
+    c = small_case(71, Hq=8, Hkv=2, ctx=(40, 300))
+    q = W.bf16_bits_to_f32(c.q) * np.float32(3.0e5)
+    q[0, 1] *= np.float32(1e-3)                     # heads of very different magnitudes
+    c.q = W.to_bf16_bits(q)
+    c.scale = 1e-5
+    run_case(c, kv="i8")
