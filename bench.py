@@ -329,12 +329,44 @@ class PrefillStep:
                 "page_size": c.page_size, "l2": "L2 flushed between steps (252 MB write outside the events)"}
 
 
-def make_step(name: str):
+def make_step(name: str, batch: int = 0, graph: bool = False):
     from paged_kv_cache_380_b200 import workloads as W
     if name == "long_ctx_split_kv_int8":
-        return DecodeStep(W.long_ctx_split_kv(), int8=True)
-    case = W.WORKLOADS[name]()
+        step = DecodeStep(W.long_ctx_split_kv(**({"batch": batch} if batch else {})), int8=True)
+        return GraphStep(step) if graph else step
+    case = W.WORKLOADS[name](**({"batch": batch} if batch else {}))
+    if graph and case.kind == "decode":
+        return GraphStep(DecodeStep(case))
     return PrefillStep(case) if case.kind == "prefill" else DecodeStep(case)
+
+
+class GraphStep:
+    """A DecodeStep replayed as one captured CUDA graph (append + decode + merge)."""
+
+    def __init__(self, inner):
+        from paged_kv_cache_380_b200.graph import DecodeStepGraph
+        self.inner = inner
+        for k in ("case", "kind", "int8", "has_new", "decode_bytes", "write_bytes", "work", "units", "launches",
+                  "splits", "split_tokens"):
+            setattr(self, k, getattr(inner, k))
+        kw = dict(k_scales=inner.ks, v_scales=inner.vs)
+        if inner.has_new:
+            kw.update(k_new=inner.k_new, v_new=inner.v_new, slot_mapping=inner.slots)
+        self.g = DecodeStepGraph(inner.q, inner.kp, inner.vp, inner.bt, inner.cl, inner.case.scale, out=inner.out, **kw)
+        self.out = inner.out
+
+    def run(self, ev=None):
+        if ev is not None:
+            ev[0].record()
+        self.g.replay()
+        if ev is not None:
+            ev[1].record()
+
+    def host_io(self):
+        return self.inner.host_io()
+
+    def config(self):
+        return dict(self.inner.config(), cuda_graph=True)
 
 
 # ---- the GPU arm ------------------------------------------------------------------------
@@ -451,7 +483,7 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
     from paged_kv_cache_380_b200 import ops
     ops.load()
-    step = make_step(args.workload)
+    step = make_step(args.workload, args.batch, args.graph)
     K, W = args.steps, max(3, args.warmup)
     for _ in range(W):
         if hasattr(step, "before_step"):
@@ -515,7 +547,8 @@ def run_ours(args):
                   else {"rows_per_s": round(units / (elapsed / 1e3), 1)}),
         "roofline": {"bound": bound, "achieved": round(achieved, 3), "peak": peak, "unit": runit,
                      "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "kernel": ("decode call (main kernel + split-KV merge)" if step.kind == "decode"
+                     "kernel": ("graph replay (append + decode + merge)" if args.graph else
+                                "decode call (main kernel + split-KV merge)" if step.kind == "decode"
                                 else "prefill kernel"),
                      "kernel_ms": round(dom_avg_ms, 5), "peak_source": f"{peak_src} (MEASURED_PEAKS.json)"
                      if peak_src == "measured" else "fallback"},
@@ -601,6 +634,9 @@ def main(argv=None):
                     choices=["tiny_decode_f32", "llama2_7b_mha_decode", "llama2_70b_gqa_decode",
                              "long_ctx_split_kv", "long_ctx_split_kv_int8", "chunked_prefill_shared_prefix"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="decode workloads: replay the step as one captured CUDA graph")
+    ap.add_argument("--batch", type=int, default=0, help="override the batch size of a decode workload")
     ap.add_argument("--cpu-seconds", type=float, default=20.0, help="CPU-baseline sample budget")
     ap.add_argument("--ref-seqs", type=int, default=4, help="reference arm: sequences per step (decode)")
     ap.add_argument("--ref-items", type=int, default=512, help="reference arm: (row, head) items per step")
