@@ -49,9 +49,9 @@ def build(force: bool = False, src: str = _SRC, out: str = _LIB) -> str:
 def _open(path):
     lib = ctypes.CDLL(path)
     P, I, I64, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
-    lib.oracle_decode.argtypes = [P, I, P, P, I, P, P, P, P, D, I, I, I, I, I, I, I64,
+    lib.oracle_decode.argtypes = [P, I, P, P, I, P, P, P, P, D, I, I, I, I, I, I, I, I64,
                                   P, I64, P, P]
-    lib.oracle_prefill.argtypes = [P, I, P, P, I, P, P, P, P, P, I, D, I, I, I, I, I, I,
+    lib.oracle_prefill.argtypes = [P, I, P, P, I, P, P, P, P, P, I, D, I, I, I, I, I, I, I,
                                    I64, P, I64, P, P]
     lib.oracle_kv_cache_write.argtypes = [P, P, P, I64, P, P, I64, I64]
     lib.oracle_quantize_int8.argtypes = [P, I, I64, I, P, P]
@@ -181,12 +181,13 @@ def _sel(sel):
 
 
 def decode(q, q_tag, k_pages, v_pages, kv_tag, block_tables, context_lens, scale,
-           k_scales=None, v_scales=None, items=None, return_lse=False):
+           k_scales=None, v_scales=None, items=None, return_lse=False, window=0):
     """fp64 decode attention: one query row per sequence.
 
     q [B, Hq, D]; pools [P, ps, Hkv, D]; block_tables int32 [B, MP];
     context_lens int32 [B].  ``items`` selects flat (b*Hq + h) rows; the
-    result is then [len(items), D], else [B, Hq, D].
+    result is then [len(items), D], else [B, Hq, D].  ``window`` > 0 keeps only
+    the last ``window`` keys (local attention).
     """
     q = _typed(q, q_tag)
     kp = _typed(k_pages, kv_tag)
@@ -206,7 +207,7 @@ def decode(q, q_tag, k_pages, v_pages, kv_tag, block_tables, context_lens, scale
     out = np.zeros((n_out, D), dtype=np.float64)
     lse = np.zeros(n_out, dtype=np.float64)
     _check(_load().oracle_decode(_ptr(q), DTYPES[q_tag], _ptr(kp), _ptr(vp), DTYPES[kv_tag],
-                                 _ptr(ks), _ptr(vs), _ptr(bt), _ptr(cl), float(scale), B, Hq, Hkv,
+                                 _ptr(ks), _ptr(vs), _ptr(bt), _ptr(cl), float(scale), int(window), B, Hq, Hkv,
                                  D, ps, bt.shape[1], P, _ptr(sel), n_sel, _ptr(out), _ptr(lse)))
     if sel is None:
         out = out.reshape(B, Hq, D)
@@ -215,7 +216,7 @@ def decode(q, q_tag, k_pages, v_pages, kv_tag, block_tables, context_lens, scale
 
 
 def prefill(q, q_tag, k_pages, v_pages, kv_tag, block_tables, q_start, context_lens, causal,
-            scale, k_scales=None, v_scales=None, items=None, return_lse=False):
+            scale, k_scales=None, v_scales=None, items=None, return_lse=False, window=0):
     """fp64 chunked-prefill attention over packed query rows q [Ttot, Hq, D].
 
     Rows q_start[b]..q_start[b+1]-1 belong to sequence b at absolute
@@ -242,7 +243,7 @@ def prefill(q, q_tag, k_pages, v_pages, kv_tag, block_tables, q_start, context_l
     lse = np.zeros(n_out, dtype=np.float64)
     _check(_load().oracle_prefill(_ptr(q), DTYPES[q_tag], _ptr(kp), _ptr(vp), DTYPES[kv_tag],
                                   _ptr(ks), _ptr(vs), _ptr(bt), _ptr(qs), _ptr(cl),
-                                  1 if causal else 0, float(scale), B, Hq, Hkv, D, ps,
+                                  1 if causal else 0, float(scale), int(window), B, Hq, Hkv, D, ps,
                                   bt.shape[1], P, _ptr(sel), n_sel, _ptr(out), _ptr(lse)))
     if sel is None:
         out = out.reshape(T, Hq, D)

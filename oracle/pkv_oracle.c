@@ -34,6 +34,10 @@
  *   - chunked prefill: a chunk of n query rows of a sequence with context
  *     length ctx sits at absolute positions ctx-n .. ctx-1 (bottom-right
  *     alignment); with causal masking row r attends keys 0 .. ctx-n+r.
+ *   - local (sliding-window) attention, the window_size argument of the
+ *     attention call in [KVFA] §5.1 ("局部注意力"): with window w > 0 a query at
+ *     position pos only sees keys pos-w+1 .. pos (keys below 0 do not exist);
+ *     w <= 0 means no window.  Decode's query sits at pos = ctx-1.
  *   - symmetric INT8 quantisation of a K/V row ([SYS] §3.2 "量化压缩的工程实践",
  *     bits = 8, one group = one (token, KV head) row):  a = max|x| (fp32),
  *     scale = fp16(a / 127) (round to nearest even), code =
@@ -203,11 +207,12 @@ static double or_kv(const or_cache* c, int is_v, int b, int i, int kvh, int d, i
     return x;
 }
 
-/* One query row (D values already in qd) against keys 0..nkeys-1 of sequence
- * b, KV head kvh.  Two-pass softmax in fp64. */
-static int or_attend(const or_cache* c, const double* qd, int b, int kvh, int nkeys,
+/* One query row (D values already in qd) against keys k_lo..k_hi-1 of
+ * sequence b, KV head kvh.  Two-pass softmax in fp64. */
+static int or_attend(const or_cache* c, const double* qd, int b, int kvh, int k_lo, int k_hi,
                      double scale, double* s, double* out, double* lse) {
     int D = c->head_dim, bad = 0;
+    int nkeys = k_hi - k_lo;
     if (nkeys <= 0) {
         for (int d = 0; d < D; ++d) out[d] = 0.0;
         *lse = -INFINITY;
@@ -215,7 +220,7 @@ static int or_attend(const or_cache* c, const double* qd, int b, int kvh, int nk
     }
     for (int i = 0; i < nkeys; ++i) {
         double dot = 0.0;
-        for (int d = 0; d < D; ++d) dot += qd[d] * or_kv(c, 0, b, i, kvh, d, &bad);
+        for (int d = 0; d < D; ++d) dot += qd[d] * or_kv(c, 0, b, k_lo + i, kvh, d, &bad);
         s[i] = scale * dot;
     }
     double m = s[0];
@@ -224,7 +229,7 @@ static int or_attend(const or_cache* c, const double* qd, int b, int kvh, int nk
     for (int i = 0; i < nkeys; ++i) { s[i] = exp(s[i] - m); L += s[i]; }
     for (int d = 0; d < D; ++d) {
         double acc = 0.0;
-        for (int i = 0; i < nkeys; ++i) acc += s[i] * or_kv(c, 1, b, i, kvh, d, &bad);
+        for (int i = 0; i < nkeys; ++i) acc += s[i] * or_kv(c, 1, b, k_lo + i, kvh, d, &bad);
         out[d] = acc / L;
     }
     *lse = m + log(L);
@@ -250,7 +255,7 @@ static int or_check_common(int num_seqs, int Hq, int Hkv, int D, int ps, int mp,
  */
 int oracle_decode(const void* q, int q_dtype, const void* k_pages, const void* v_pages,
                   int kv_dtype, const uint16_t* k_scales, const uint16_t* v_scales,
-                  const int32_t* block_tables, const int32_t* context_lens, double scale,
+                  const int32_t* block_tables, const int32_t* context_lens, double scale, int window,
                   int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int page_size,
                   int max_pages_per_seq, int64_t num_pages,
                   const int64_t* sel_items, int64_t n_sel, double* out, double* lse) {
@@ -289,8 +294,9 @@ int oracle_decode(const void* q, int q_dtype, const void* k_pages, const void* v
             for (int d = 0; d < head_dim; ++d)
                 qd[d] = or_elem(q, q_dtype, item * head_dim + d);
             double l;
-            int r = or_attend(&c, qd, b, h / G, context_lens[b], scale, s,
-                              out + it * head_dim, &l);
+            int ctx = context_lens[b];
+            int k_lo = (window > 0 && ctx - window > 0) ? ctx - window : 0;
+            int r = or_attend(&c, qd, b, h / G, k_lo, ctx, scale, s, out + it * head_dim, &l);
             if (lse) lse[it] = l;
             if (r) {
 #pragma omp critical
@@ -313,7 +319,7 @@ int oracle_decode(const void* q, int q_dtype, const void* k_pages, const void* v
 int oracle_prefill(const void* q, int q_dtype, const void* k_pages, const void* v_pages,
                    int kv_dtype, const uint16_t* k_scales, const uint16_t* v_scales,
                    const int32_t* block_tables, const int32_t* q_start,
-                   const int32_t* context_lens, int causal, double scale,
+                   const int32_t* context_lens, int causal, double scale, int window,
                    int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int page_size,
                    int max_pages_per_seq, int64_t num_pages,
                    const int64_t* sel_items, int64_t n_sel, double* out, double* lse) {
@@ -361,11 +367,12 @@ int oracle_prefill(const void* q, int q_dtype, const void* k_pages, const void* 
             int n = q_start[b + 1] - q_start[b], ctx = context_lens[b];
             int r = (int)(t - q_start[b]);
             int pos = ctx - n + r;
-            int nkeys = causal ? pos + 1 : ctx;
+            int k_hi = causal ? pos + 1 : ctx;
+            int k_lo = (window > 0 && pos - window + 1 > 0) ? pos - window + 1 : 0;
             for (int d = 0; d < head_dim; ++d)
                 qd[d] = or_elem(q, q_dtype, item * head_dim + d);
             double l;
-            int rr = or_attend(&c, qd, b, h / G, nkeys, scale, s, out + it * head_dim, &l);
+            int rr = or_attend(&c, qd, b, h / G, k_lo, k_hi, scale, s, out + it * head_dim, &l);
             if (lse) lse[it] = l;
             if (rr) {
 #pragma omp critical

@@ -31,6 +31,8 @@ MUTANTS = [
     ("f16_round_truncates", "double r = rint(ldexp(a, 10 - E));", "double r = floor(ldexp(a, 10 - E));"),
     ("bf16_shift", "(uint32_t)b << 16", "(uint32_t)b << 15"),
     ("scatter_swaps_kv", "(const char*)v + t * row_bytes", "(const char*)k + t * row_bytes"),
+    ("window_off_by_one", "pos - window + 1 > 0) ? pos - window + 1 : 0", "pos - window > 0) ? pos - window : 0"),
+    ("decode_window_ignored", "(window > 0 && ctx - window > 0) ? ctx - window : 0", "0"),
 ]
 
 CHECKS = [
@@ -56,6 +58,9 @@ CHECKS = [
     pins.test_scatter_matches_fancy_index_assignment,
     pins.test_f16_widening_and_rounding_match_numpy,
     pins.test_bf16_widening_matches_torch_for_all_patterns,
+    pins.test_window_covering_the_context_equals_no_window,
+    pins.test_window_one_returns_the_own_value,
+    lambda: pins.test_window_matches_sdpa_band_mask(3),
 ]
 
 

@@ -411,3 +411,44 @@ def test_scatter_out_of_range_slot_is_an_error():
     with pytest.raises(ValueError):
         oracle.kv_cache_write(np.ones((1, 1, 8), np.uint16), np.ones((1, 1, 8), np.uint16),
                               np.array([8]), kp, vp)
+
+
+# ---- local (sliding-window) attention ------------------------------------------
+
+def test_window_covering_the_context_equals_no_window():
+    rng = np.random.default_rng(30)
+    c = random_paged(rng, ctx=(5, 8, 13))
+    assert np.array_equal(run_decode(c, 0.5, window=13), run_decode(c, 0.5))
+    c2, q, qs, ctx = _prefill_case(rng)
+    a = oracle.prefill(q, "f64", c2["k"], c2["v"], "f64", c2["bt"], qs, ctx, True, 0.5, window=int(ctx.max()))
+    b_ = oracle.prefill(q, "f64", c2["k"], c2["v"], "f64", c2["bt"], qs, ctx, True, 0.5)
+    assert np.array_equal(a, b_)
+
+
+def test_window_one_returns_the_own_value():
+    rng = np.random.default_rng(31)
+    c = random_paged(rng, ctx=(5, 8, 13))
+    out = run_decode(c, 0.9, window=1)
+    for b in range(3):
+        v_last = gather(c["v"], c["bt"][b], c["ps"], int(c["ctx"][b]))[-1]
+        for h in range(4):
+            assert np.array_equal(out[b, h], v_last[h // 2])
+
+
+@pytest.mark.parametrize("window", [1, 3, 6])
+def test_window_matches_sdpa_band_mask(window):
+    rng = np.random.default_rng(32)
+    c, q, qs, ctx = _prefill_case(rng)
+    out = oracle.prefill(q, "f64", c["k"], c["v"], "f64", c["bt"], qs, ctx, True, 0.35, window=window)
+    Hq, Hkv = 4, 2
+    for b in range(len(ctx)):
+        n, L = int(qs[b + 1] - qs[b]), int(ctx[b])
+        K = torch.from_numpy(gather(c["k"], c["bt"][b], c["ps"], L)).permute(1, 0, 2).repeat_interleave(2, 0)
+        V = torch.from_numpy(gather(c["v"], c["bt"][b], c["ps"], L)).permute(1, 0, 2).repeat_interleave(2, 0)
+        Q = torch.from_numpy(q[qs[b]:qs[b + 1]]).permute(1, 0, 2)
+        pos = (L - n + torch.arange(n))[:, None]
+        key = torch.arange(L)[None, :]
+        mask = (key <= pos) & (key > pos - window)
+        ref = torch.nn.functional.scaled_dot_product_attention(Q, K, V, attn_mask=mask, scale=0.35)
+        got = torch.from_numpy(out[qs[b]:qs[b + 1]]).permute(1, 0, 2)
+        assert (got - ref).abs().max().item() < 1e-12
