@@ -62,7 +62,8 @@ enum {
     PKV_ERR_WORKSPACE = -3,     /* workspace missing or too small */
     PKV_ERR_CUDA = -4,          /* a CUDA runtime call failed (launch, device query) */
     PKV_ERR_DEVICE_RANGE = -5,  /* device saw an out-of-range page, slot or length */
-    PKV_ERR_DEVICE_TIMEOUT = -6 /* a bounded device wait gave up (pipeline stalled) */
+    PKV_ERR_DEVICE_TIMEOUT = -6, /* a bounded device wait gave up (pipeline stalled) */
+    PKV_ERR_OUT_OF_PAGES = -7    /* block manager: not enough free pages (nothing changed) */
 };
 
 /* Static description of a status code (thread-safe, never NULL). */
@@ -220,6 +221,56 @@ int pkv_paged_attention_prefill(const void* q, const void* k_pages, const void* 
                                 int num_q_heads, int num_kv_heads, int head_dim,
                                 int page_size, int max_pages_per_seq, int64_t num_pages,
                                 pkv_dtype dtype, pkv_stream_t stream);
+
+/*
+ * Host-side block manager for the paged pool (pure host code, thread-safe, no
+ * CUDA call).  GPU memory is cut into fixed-size pages handed out on demand
+ * and released whole ([KVFA] §4.1 块级内存池); sequences that share a prompt
+ * share its pages with reference counts ([KVFA] §4.1 零拷贝共享, [SYS] §3.1);
+ * each sequence's page table maps logical to physical pages ([FAPKV] §3.2) and
+ * freeing a sequence deletes its table entry (the leak fix of [FAPKV] §5.2).
+ *   create:   num_pages physical pages of page_size tokens, at most
+ *             max_pages_per_seq pages per sequence; NULL on bad arguments.
+ *   add_sequence: a new empty sequence; its id is written to *seq_id_out.
+ *   fork:     a child sequence sharing every page of the parent (refcount + 1).
+ *   append:   reserve slots for num_tokens new tokens at the end of `seq`
+ *             (slots_out[num_tokens], slot = page * page_size + offset, ready for
+ *             pkv_kv_cache_write).  If the last page is shared and not full it is
+ *             first replaced by a private page (copy-on-write): the pair is
+ *             returned in copy_src[0] / copy_dst[0] (arrays of >= 1 entry) with
+ *             *num_copies = 1, and the caller must run pkv_copy_pages before
+ *             writing.  PKV_ERR_OUT_OF_PAGES (or INVALID_ARG past
+ *             max_pages_per_seq) leaves the manager unchanged.
+ *   free_sequence: drop the sequence's page references and delete its entry;
+ *             pages whose count reaches zero return to the free pool.  Freeing an
+ *             unknown or already freed id is PKV_ERR_INVALID_ARG.
+ *   block_tables: export int32 [num_seqs][max_pages_per_seq] tables (-1 past
+ *             the last page) and context lengths for the attention calls.
+ */
+typedef struct pkv_block_manager pkv_block_manager;
+pkv_block_manager* pkv_bm_create(int64_t num_pages, int page_size, int max_pages_per_seq);
+void pkv_bm_destroy(pkv_block_manager* bm);
+int pkv_bm_add_sequence(pkv_block_manager* bm, int64_t* seq_id_out);
+int pkv_bm_fork(pkv_block_manager* bm, int64_t parent, int64_t* child_out);
+int pkv_bm_append(pkv_block_manager* bm, int64_t seq, int num_tokens, int64_t* slots_out,
+                  int32_t* copy_src, int32_t* copy_dst, int* num_copies);
+int pkv_bm_free_sequence(pkv_block_manager* bm, int64_t seq);
+int pkv_bm_block_tables(pkv_block_manager* bm, const int64_t* seq_ids, int num_seqs,
+                        int32_t* table_out, int32_t* context_lens_out);
+int64_t pkv_bm_num_free_pages(pkv_block_manager* bm);
+int pkv_bm_page_refcount(pkv_block_manager* bm, int32_t page);   /* or PKV_ERR_INVALID_ARG */
+int pkv_bm_num_sequences(pkv_block_manager* bm);
+
+/*
+ * Device copy of whole pages for copy-on-write: page src[i] of the K and V
+ * pools is copied to page dst[i] (page_bytes = page_size * num_kv_heads *
+ * head_dim * element size; for INT8 pools call it again on the scale pools
+ * with their page size in bytes).  src/dst are device int32 arrays of
+ * num_copies entries; an out-of-range page is skipped and recorded in the
+ * device status word.  Bit-exact.
+ */
+int pkv_copy_pages(void* k_pages, void* v_pages, const int32_t* src, const int32_t* dst,
+                   int num_copies, int64_t page_bytes, int64_t num_pages, pkv_stream_t stream);
 
 /*
  * Synchronises `stream`, then reads and clears the device status word of the

@@ -97,6 +97,8 @@ int from_cuda(cudaError_t e) { return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA; 
 
 }  // namespace
 
+DeviceStatus* device_status_ptr() { return status_ptr(); }
+
 cudaError_t ensure_dynamic_smem(const void* kernel, int bytes) {
     static std::mutex mu;
     static std::set<std::pair<const void*, int>> done;
@@ -125,6 +127,7 @@ const char* pkv_error_string(int code) {
     case PKV_ERR_CUDA: return "a CUDA runtime call failed";
     case PKV_ERR_DEVICE_RANGE: return "device saw an out-of-range page, slot or length (access skipped)";
     case PKV_ERR_DEVICE_TIMEOUT: return "a bounded device wait gave up";
+    case PKV_ERR_OUT_OF_PAGES: return "the block manager has no free page left";
     default: return "unknown pagedkv status";
     }
 }

@@ -8,6 +8,9 @@
 
 namespace pkv {
 
+// Device address of this device's status word (set up on first use).
+DeviceStatus* device_status_ptr();
+
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel, device).
 cudaError_t ensure_dynamic_smem(const void* kernel, int bytes);
 

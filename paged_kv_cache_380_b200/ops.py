@@ -27,7 +27,9 @@ _DT = {torch.float32: PKV_F32, torch.bfloat16: PKV_BF16, torch.float16: PKV_F16,
 EXPORTS = ("pkv_error_string", "pkv_kv_cache_write", "pkv_kv_cache_write_quant", "pkv_paged_attention_decode",
            "pkv_decode_workspace_size", "pkv_decode_plan", "pkv_paged_attention_decode_noalloc",
            "pkv_paged_attention_prefill",
-           "pkv_get_device_status")
+           "pkv_get_device_status", "pkv_bm_create", "pkv_bm_destroy", "pkv_bm_add_sequence", "pkv_bm_fork",
+           "pkv_bm_append", "pkv_bm_free_sequence", "pkv_bm_block_tables", "pkv_bm_num_free_pages",
+           "pkv_bm_page_refcount", "pkv_bm_num_sequences", "pkv_copy_pages")
 
 
 class PagedKVError(RuntimeError):
@@ -68,6 +70,23 @@ def load(path: str = _LIB_PATH):
         lib.pkv_paged_attention_prefill.restype = I
         lib.pkv_get_device_status.argtypes = [P, ctypes.POINTER(I64)]
         lib.pkv_get_device_status.restype = I
+        lib.pkv_bm_create.argtypes = [I64, I, I]
+        lib.pkv_bm_create.restype = P
+        lib.pkv_bm_destroy.argtypes = [P]
+        lib.pkv_bm_destroy.restype = None
+        lib.pkv_bm_add_sequence.argtypes = [P, ctypes.POINTER(I64)]
+        lib.pkv_bm_fork.argtypes = [P, I64, ctypes.POINTER(I64)]
+        lib.pkv_bm_append.argtypes = [P, I64, I, P, P, P, ctypes.POINTER(I)]
+        lib.pkv_bm_free_sequence.argtypes = [P, I64]
+        lib.pkv_bm_block_tables.argtypes = [P, P, I, P, P]
+        lib.pkv_bm_num_free_pages.argtypes = [P]
+        lib.pkv_bm_num_free_pages.restype = I64
+        lib.pkv_bm_page_refcount.argtypes = [P, ctypes.c_int32]
+        lib.pkv_bm_num_sequences.argtypes = [P]
+        lib.pkv_copy_pages.argtypes = [P, P, P, P, I, I64, I64, P]
+        for f in (lib.pkv_bm_add_sequence, lib.pkv_bm_fork, lib.pkv_bm_append, lib.pkv_bm_free_sequence,
+                  lib.pkv_bm_block_tables, lib.pkv_bm_page_refcount, lib.pkv_bm_num_sequences, lib.pkv_copy_pages):
+            f.restype = I
         _lib = lib
     return _lib
 
@@ -227,3 +246,74 @@ def device_status(stream=None):
     detail = ctypes.c_int64(-1)
     code = load().pkv_get_device_status(_stream(stream), ctypes.byref(detail))
     return int(code), int(detail.value)
+
+
+def copy_pages(k_pages, v_pages, src, dst, *, stream=None) -> None:
+    """Copy whole pages src[i] -> dst[i] (int32 CUDA tensors) of both pools."""
+    _cuda(k_pages, v_pages, src, dst)
+    P = k_pages.shape[0]
+    page_bytes = k_pages[0].numel() * k_pages.element_size()
+    _check(load().pkv_copy_pages(_ptr(k_pages), _ptr(v_pages), _ptr(src), _ptr(dst), int(src.numel()), page_bytes,
+                                 P, _stream(stream)), "copy_pages")
+
+
+class BlockManager:
+    """Host-side page allocator of the C library: refcounted pages, fork with
+    shared pages, copy-on-write on append, release that deletes the table entry."""
+
+    def __init__(self, num_pages: int, page_size: int, max_pages_per_seq: int):
+        self._lib = load()
+        self._h = self._lib.pkv_bm_create(int(num_pages), int(page_size), int(max_pages_per_seq))
+        if not self._h:
+            raise ValueError("invalid block manager sizes")
+        self.page_size, self.max_pages_per_seq = page_size, max_pages_per_seq
+
+    def __del__(self):
+        if getattr(self, "_h", None):
+            self._lib.pkv_bm_destroy(self._h)
+            self._h = None
+
+    def add_sequence(self) -> int:
+        out = ctypes.c_int64()
+        _check(self._lib.pkv_bm_add_sequence(self._h, ctypes.byref(out)), "bm_add_sequence")
+        return out.value
+
+    def fork(self, parent: int) -> int:
+        out = ctypes.c_int64()
+        _check(self._lib.pkv_bm_fork(self._h, int(parent), ctypes.byref(out)), "bm_fork")
+        return out.value
+
+    def append(self, seq: int, num_tokens: int):
+        """Returns (slots int64 numpy [num_tokens], copies [(src, dst)])."""
+        import numpy as np
+        slots = np.empty(max(num_tokens, 1), dtype=np.int64)
+        src, dst, n = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int()
+        _check(self._lib.pkv_bm_append(self._h, int(seq), int(num_tokens), slots.ctypes.data_as(ctypes.c_void_p),
+                                       ctypes.byref(src), ctypes.byref(dst), ctypes.byref(n)), "bm_append")
+        return slots[:num_tokens], ([(src.value, dst.value)] if n.value else [])
+
+    def free(self, seq: int) -> None:
+        _check(self._lib.pkv_bm_free_sequence(self._h, int(seq)), "bm_free_sequence")
+
+    def block_tables(self, seq_ids):
+        """(int32 [len(seq_ids), max_pages_per_seq] tables, int32 context lengths)."""
+        import numpy as np
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        table = np.empty((ids.shape[0], self.max_pages_per_seq), dtype=np.int32)
+        lens = np.empty(ids.shape[0], dtype=np.int32)
+        _check(self._lib.pkv_bm_block_tables(self._h, ids.ctypes.data_as(ctypes.c_void_p), ids.shape[0],
+                                             table.ctypes.data_as(ctypes.c_void_p),
+                                             lens.ctypes.data_as(ctypes.c_void_p)), "bm_block_tables")
+        return table, lens
+
+    def num_free_pages(self) -> int:
+        return int(self._lib.pkv_bm_num_free_pages(self._h))
+
+    def refcount(self, page: int) -> int:
+        r = self._lib.pkv_bm_page_refcount(self._h, int(page))
+        if r < 0:
+            raise PagedKVError(r, "bm_page_refcount")
+        return r
+
+    def num_sequences(self) -> int:
+        return int(self._lib.pkv_bm_num_sequences(self._h))
