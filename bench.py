@@ -193,11 +193,11 @@ class DecodeStep:
 
     kind = "decode"
 
-    def __init__(self, case, int8: bool = False):
+    def __init__(self, case, int8: bool = False, window: int = 0):
         import numpy as np
         import torch
         from paged_kv_cache_380_b200 import ops
-        self.case, self.int8 = case, int8
+        self.case, self.int8, self.window = case, int8, window
         tag = case.dtype
         B, Hq, D = case.q.shape
         P, ps, Hkv, _ = case.k_pages.shape
@@ -231,8 +231,10 @@ class DecodeStep:
         self.ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
         qelem = 4 if tag == "f32" else 2
         ctx = case.context_lens.astype(np.int64)
+        if window > 0:
+            ctx = np.minimum(ctx, window)                      # keys a windowed query reads
         pages = int(np.sum((ctx + ps - 1) // ps))
-        # algorithmic bytes: every cached K/V element read once (+ its scale for INT8),
+        # algorithmic bytes: every attended K/V element read once (+ its scale for INT8),
         # q read, out written, block-table entries and context lengths read
         self.decode_bytes = (int(ctx.sum()) * Hkv * (2 * D * elem + 2 * scale_bytes)
                              + 2 * B * Hq * D * qelem + pages * 4 + B * 4)
@@ -252,7 +254,7 @@ class DecodeStep:
         if ev is not None:
             ev[0].record()
         ops.paged_attention_decode(self.q, self.kp, self.vp, self.bt, self.cl, self.case.scale, self.out,
-                                   k_scales=self.ks, v_scales=self.vs, workspace=self.ws)
+                                   k_scales=self.ks, v_scales=self.vs, workspace=self.ws, window=self.window)
         if ev is not None:
             ev[1].record()
 
@@ -270,6 +272,7 @@ class DecodeStep:
         return {"workload": c.name + ("_int8" if self.int8 else ""), "batch": B, "num_q_heads": Hq,
                 "num_kv_heads": c.num_kv_heads, "head_dim": D, "page_size": c.page_size,
                 "kv_dtype": "i8" if self.int8 else c.dtype, "mean_context": float(c.context_lens.mean()),
+                "window": self.window,
                 "num_pages": c.num_pages, "splits": self.splits, "split_tokens": self.split_tokens,
                 "new_tokens_written": int(c.k_new.shape[0]) if self.has_new else 0,
                 "l2": ("inputs larger than L2 (%.2f GB read per step vs 126 MB L2)" % (self.work / 1e9))}
@@ -280,10 +283,10 @@ class PrefillStep:
 
     kind = "prefill"
 
-    def __init__(self, case):
+    def __init__(self, case, window: int = 0):
         import numpy as np
         import torch
-        self.case = case
+        self.case, self.window = case, window
         tag = case.dtype
         self.q = dev(case.q, tag)
         self.kp, self.vp = dev(case.k_pages, tag), dev(case.v_pages, tag)
@@ -294,8 +297,11 @@ class PrefillStep:
         Hq, D = case.num_q_heads, case.head_dim
         n = np.diff(case.q_start).astype(np.int64)
         ctx = case.context_lens.astype(np.int64)
-        # keys attended per (row, head): ctx - n + r + 1 for r < n
-        keys = int(np.sum(n * (ctx - n) + n * (n + 1) // 2))
+        # keys attended per (row, head): ctx - n + r + 1 for r < n (at most `window` of them)
+        if window > 0:
+            keys = int(sum(np.minimum(np.arange(c - k + 1, c + 1), window).sum() for k, c in zip(n, ctx)))
+        else:
+            keys = int(np.sum(n * (ctx - n) + n * (n + 1) // 2))
         self.work = 4.0 * D * Hq * keys           # flops per step (QK^T and PV, 2 flops per MAC)
         self.units = int(n.sum())                  # query rows processed
         self.launches = 2
@@ -310,7 +316,7 @@ class PrefillStep:
         if ev is not None:
             ev[0].record()
         ops.paged_attention_prefill(self.q, self.kp, self.vp, self.bt, self.qs, self.cl, True, self.case.scale,
-                                    self.out, max_q_len=self.max_q)
+                                    self.out, max_q_len=self.max_q, window=self.window)
         if ev is not None:
             ev[1].record()
 
@@ -326,18 +332,19 @@ class PrefillStep:
         return {"workload": c.name, "num_seqs": c.batch, "chunk": int(np.diff(c.q_start)[0]) if c.batch else 0,
                 "context": int(c.context_lens[0]), "shared_prefix_pages": c.meta.get("shared_pages"),
                 "num_q_heads": c.num_q_heads, "num_kv_heads": c.num_kv_heads, "head_dim": c.head_dim,
-                "page_size": c.page_size, "l2": "L2 flushed between steps (252 MB write outside the events)"}
+                "page_size": c.page_size, "window": self.window,
+                "l2": "L2 flushed between steps (252 MB write outside the events)"}
 
 
-def make_step(name: str, batch: int = 0, graph: bool = False):
+def make_step(name: str, batch: int = 0, graph: bool = False, window: int = 0):
     from paged_kv_cache_380_b200 import workloads as W
     if name == "long_ctx_split_kv_int8":
-        step = DecodeStep(W.long_ctx_split_kv(**({"batch": batch} if batch else {})), int8=True)
+        step = DecodeStep(W.long_ctx_split_kv(**({"batch": batch} if batch else {})), int8=True, window=window)
         return GraphStep(step) if graph else step
     case = W.WORKLOADS[name](**({"batch": batch} if batch else {}))
     if graph and case.kind == "decode":
-        return GraphStep(DecodeStep(case))
-    return PrefillStep(case) if case.kind == "prefill" else DecodeStep(case)
+        return GraphStep(DecodeStep(case, window=window))
+    return PrefillStep(case, window) if case.kind == "prefill" else DecodeStep(case, window=window)
 
 
 class GraphStep:
@@ -483,7 +490,7 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
     from paged_kv_cache_380_b200 import ops
     ops.load()
-    step = make_step(args.workload, args.batch, args.graph)
+    step = make_step(args.workload, args.batch, args.graph, args.window)
     K, W = args.steps, max(3, args.warmup)
     for _ in range(W):
         if hasattr(step, "before_step"):
@@ -637,6 +644,7 @@ def main(argv=None):
     ap.add_argument("--graph", action="store_true",
                     help="decode workloads: replay the step as one captured CUDA graph")
     ap.add_argument("--batch", type=int, default=0, help="override the batch size of a decode workload")
+    ap.add_argument("--window", type=int, default=0, help="local attention: attend only the last W keys")
     ap.add_argument("--cpu-seconds", type=float, default=20.0, help="CPU-baseline sample budget")
     ap.add_argument("--ref-seqs", type=int, default=4, help="reference arm: sequences per step (decode)")
     ap.add_argument("--ref-items", type=int, default=512, help="reference arm: (row, head) items per step")

@@ -154,6 +154,21 @@ int pkv_paged_attention_decode(const void* q, const void* k_pages, const void* v
                                void* workspace, size_t workspace_bytes, int num_splits,
                                pkv_stream_t stream);
 
+/*
+ * Decode with local (sliding-window) attention: as pkv_paged_attention_decode,
+ * but with window > 0 the query (at position context_lens[b]-1) attends only
+ * its last `window` keys (the window_size of the local-attention call in [KVFA]
+ * §5.1); window <= 0 is the plain call.  Same workspace size.
+ */
+int pkv_paged_attention_decode_ex(const void* q, const void* k_pages, const void* v_pages,
+                                  const int32_t* block_tables, const int32_t* context_lens,
+                                  float scale, void* out, int num_seqs, int num_q_heads,
+                                  int num_kv_heads, int head_dim, int page_size,
+                                  int max_pages_per_seq, int64_t num_pages, pkv_dtype q_dtype,
+                                  pkv_dtype kv_dtype, const void* k_scales, const void* v_scales,
+                                  void* workspace, size_t workspace_bytes, int num_splits, int window,
+                                  pkv_stream_t stream);
+
 /* Workspace bytes pkv_paged_attention_decode needs for these arguments (0 when
  * no sequence can be split).  Pure host function, no CUDA call. */
 size_t pkv_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
@@ -165,6 +180,20 @@ size_t pkv_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads
 int pkv_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                     int page_size, int max_pages_per_seq, pkv_dtype kv_dtype, int num_splits,
                     int* splits_out, int* split_tokens_out);
+
+/*
+ * Prefill with local (sliding-window) attention: as pkv_paged_attention_prefill,
+ * but with window > 0 a query row at absolute position pos attends keys
+ * max(0, pos-window+1) .. pos (causal) or .. context_len-1 (non-causal);
+ * window <= 0 is the plain call.
+ */
+int pkv_paged_attention_prefill_ex(const void* q, const void* k_pages, const void* v_pages,
+                                   const int32_t* block_tables, const int32_t* q_start,
+                                   const int32_t* context_lens, int causal, float scale,
+                                   void* out, int num_seqs, int total_q, int max_q_len,
+                                   int num_q_heads, int num_kv_heads, int head_dim,
+                                   int page_size, int max_pages_per_seq, int64_t num_pages,
+                                   pkv_dtype dtype, int window, pkv_stream_t stream);
 
 /*
  * Decode attention without any device allocation by the caller.  The pages

@@ -208,6 +208,19 @@ int pkv_paged_attention_decode(const void* q, const void* k_pages, const void* v
                                pkv_dtype kv_dtype, const void* k_scales, const void* v_scales,
                                void* workspace, size_t workspace_bytes, int num_splits,
                                pkv_stream_t stream) {
+    return pkv_paged_attention_decode_ex(q, k_pages, v_pages, block_tables, context_lens, scale, out, num_seqs,
+                                         num_q_heads, num_kv_heads, head_dim, page_size, max_pages_per_seq,
+                                         num_pages, q_dtype, kv_dtype, k_scales, v_scales, workspace,
+                                         workspace_bytes, num_splits, 0, stream);
+}
+
+int pkv_paged_attention_decode_ex(const void* q, const void* k_pages, const void* v_pages,
+                                  const int32_t* block_tables, const int32_t* context_lens, float scale,
+                                  void* out, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                  int page_size, int max_pages_per_seq, int64_t num_pages, pkv_dtype q_dtype,
+                                  pkv_dtype kv_dtype, const void* k_scales, const void* v_scales,
+                                  void* workspace, size_t workspace_bytes, int num_splits, int window,
+                                  pkv_stream_t stream) {
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || page_size <= 0 ||
         max_pages_per_seq <= 0 || num_pages <= 0 || num_splits < 0 || !std::isfinite(scale))
         return PKV_ERR_INVALID_ARG;
@@ -258,6 +271,7 @@ int pkv_paged_attention_decode(const void* q, const void* k_pages, const void* v
     p.num_pages = num_pages;
     p.chunks_per_split = pl.chunks_per_split;
     p.max_splits = pl.splits;
+    p.window = window > 0 ? window : 0;
     p.status = st;
     return from_cuda(launch_decode(p, q_dtype, kv_dtype, reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -268,6 +282,17 @@ int pkv_paged_attention_prefill(const void* q, const void* k_pages, const void* 
                                 int num_seqs, int total_q, int max_q_len, int num_q_heads, int num_kv_heads,
                                 int head_dim, int page_size, int max_pages_per_seq, int64_t num_pages,
                                 pkv_dtype dtype, pkv_stream_t stream) {
+    return pkv_paged_attention_prefill_ex(q, k_pages, v_pages, block_tables, q_start, context_lens, causal, scale,
+                                          out, num_seqs, total_q, max_q_len, num_q_heads, num_kv_heads, head_dim,
+                                          page_size, max_pages_per_seq, num_pages, dtype, 0, stream);
+}
+
+int pkv_paged_attention_prefill_ex(const void* q, const void* k_pages, const void* v_pages,
+                                   const int32_t* block_tables, const int32_t* q_start,
+                                   const int32_t* context_lens, int causal, float scale, void* out,
+                                   int num_seqs, int total_q, int max_q_len, int num_q_heads, int num_kv_heads,
+                                   int head_dim, int page_size, int max_pages_per_seq, int64_t num_pages,
+                                   pkv_dtype dtype, int window, pkv_stream_t stream) {
     if (num_seqs < 0 || total_q < 0 || max_q_len < 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
         head_dim <= 0 || page_size <= 0 || max_pages_per_seq <= 0 || num_pages <= 0 || !std::isfinite(scale))
         return PKV_ERR_INVALID_ARG;
@@ -300,6 +325,7 @@ int pkv_paged_attention_prefill(const void* q, const void* k_pages, const void* 
     p.page_size = page_size;
     p.max_pages_per_seq = max_pages_per_seq;
     p.num_pages = num_pages;
+    p.window = window > 0 ? window : 0;
     p.status = st;
     return from_cuda(launch_prefill(p, dtype, reinterpret_cast<cudaStream_t>(stream)));
 }

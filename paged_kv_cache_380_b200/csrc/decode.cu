@@ -108,11 +108,14 @@ decode_mma_kernel(const DecodeParams p) {
             for (int i = threadIdx.x; i < G * HD; i += WARPS * 32) out[head0 * HD + i] = from_float<QT>(0.f);
         return;
     }
-    const int n_chunks = ceil_div(ctx, kChunk);
+    // keys k_lo .. ctx-1 are attended (k_lo > 0 only with a local-attention window)
+    const int k_lo = (p.window > 0 && ctx > p.window) ? ctx - p.window : 0;
+    const int c_lo = k_lo / kChunk;
+    const int n_chunks = ceil_div(ctx, kChunk) - c_lo;
     const int nsplit = ceil_div(n_chunks, p.chunks_per_split);
     if (split >= nsplit) return;
-    const int c_begin = split * p.chunks_per_split;
-    const int c_end = min(c_begin + p.chunks_per_split, n_chunks);
+    const int c_begin = c_lo + split * p.chunks_per_split;
+    const int c_end = min(c_begin + p.chunks_per_split, c_lo + n_chunks);
     const int n_mine = (c_end - c_begin > warp) ? ceil_div(c_end - c_begin - warp, WARPS) : 0;
 
     // ---- query fragments (B operand of S^T = K . Q^T), kept in registers ----
@@ -279,7 +282,7 @@ decode_mma_kernel(const DecodeParams p) {
             ks_a = scale_at(0, g); ks_b = scale_at(0, g + 8);
             vs_a = scale_at(64, g); vs_b = scale_at(64, g + 8);
         }
-        const bool va = tok0 + g < ctx, vb = tok0 + g + 8 < ctx;
+        const bool va = tok0 + g < ctx && tok0 + g >= k_lo, vb = tok0 + g + 8 < ctx && tok0 + g + 8 >= k_lo;
         uint32_t pb[NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -295,7 +298,7 @@ decode_mma_kernel(const DecodeParams p) {
                 mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
                 mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
                 mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
-                const float m_new = fmaxf(m[nt][h], mx);   // finite: token tok0 is in the context
+                const float m_new = fmaxf(m[nt][h], mx);   // finite: every chunk holds an attended token
                 const float corr = ptx::ex2(m[nt][h] - m_new);
                 m[nt][h] = m_new;
                 pr[h] = ptx::ex2(x[h] - m_new);
@@ -428,7 +431,8 @@ __global__ void __launch_bounds__(kCombineWarps * 32) decode_combine_kernel(cons
     const int b = gw / p.num_q_heads;
     const int ctx = __ldg(p.context_lens + b);
     if (ctx <= 0 || ctx > p.max_pages_per_seq * p.page_size) return;
-    const int ns = ceil_div(ceil_div(ctx, kChunk), p.chunks_per_split);
+    const int k_lo = (p.window > 0 && ctx > p.window) ? ctx - p.window : 0;
+    const int ns = ceil_div(ceil_div(ctx, kChunk) - k_lo / kChunk, p.chunks_per_split);
     if (ns <= 1) return;
     const float* lse = p.lse_part + static_cast<size_t>(gw) * p.max_splits;
     const float* op = p.o_part + static_cast<size_t>(gw) * p.max_splits * HD;
@@ -497,7 +501,8 @@ __global__ void __launch_bounds__(128) decode_f32_kernel(const DecodeParams p) {
 #pragma unroll
         for (int j = 0; j < E; ++j) { qv[j] = q[h * HD + lane + 32 * j]; acc[j] = 0.f; }
         float mx = -INFINITY, l = 0.f;
-        for (int t = 0; t < ctx; ++t) {
+        const int k_lo = (p.window > 0 && ctx > p.window) ? ctx - p.window : 0;
+        for (int t = k_lo; t < ctx; ++t) {
             const int page = __ldg(bt + t / ps);
             if (page < 0 || page >= p.num_pages) {
                 if (lane == 0) record_error(p.status, PKV_ERR_DEVICE_RANGE, page);

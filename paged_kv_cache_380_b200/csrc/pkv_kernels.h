@@ -44,6 +44,7 @@ struct DecodeParams {
     int64_t num_pages;
     int chunks_per_split;  // 16-token chunks per partition
     int max_splits;        // partitions the workspace holds (1 = no workspace)
+    int window;            // > 0: only the last `window` keys are attended (local attention)
     DeviceStatus* status;
 };
 
@@ -64,6 +65,7 @@ struct PrefillParams {
     int num_seqs, total_q, max_q_len, num_q_heads, num_kv_heads, head_dim, page_size;
     int max_pages_per_seq;
     int64_t num_pages;
+    int window;            // > 0: a query at pos sees keys pos-window+1 .. pos only
     DeviceStatus* status;
 };
 

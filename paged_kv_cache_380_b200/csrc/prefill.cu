@@ -154,18 +154,16 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
     }
     const int last_row = min(r0 + BM, n) - 1;
     const int max_key = p.causal ? ctx - n + last_row : ctx - 1;
-    const int n_tiles = max_key / BN + 1;
     const int min_lim = p.causal ? ctx - n + r0 : ctx - 1;      // every row of the tile sees keys <= this
-    // Tiles every row sees in full are visited in a rotated order that differs
-    // between the CTAs reading the same pages (query heads of one KV head, and
-    // sequences sharing a prefix), so concurrent CTAs do not all fetch the same
-    // lines at once; masked (diagonal / last) tiles follow in order.
-#ifndef PKV_PREFILL_ROTATE
-#define PKV_PREFILL_ROTATE 1
-#endif
-    const int n_full = min((min_lim + 1) / BN, n_tiles);
-    const int rot = (PKV_PREFILL_ROTATE && n_full > 1) ? (h * 3 + b * 5) % n_full : 0;
-    auto tile_of = [&](int j) { return j < n_full ? (j + rot) % n_full : j; };
+    // Local attention (window w > 0): a row at position pos sees keys pos-w+1 .. pos,
+    // so the tile's key range starts at the first row's lower bound, and keys below
+    // the last row's lower bound need the lower-edge mask.
+    const int w = p.window;
+    const int key_lo = w > 0 ? max(0, ctx - n + r0 - w + 1) : 0;
+    const int lo_mask = w > 0 ? max(0, ctx - n + last_row - w + 1) : 0;
+    const int t_first = key_lo / BN;
+    const int n_tiles = max_key / BN + 1 - t_first;
+    auto tile_of = [&](int j) { return t_first + j; };
 
     const Bars bars{sbase + kSmemBar};
     // Page indices, 4 tiles (32 groups of 16 keys) per batch: lane i of batch k holds the
@@ -326,6 +324,7 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
         float* red = reinterpret_cast<float*>(smem + kSmemRed);     // [2 bufs][2 halves][BM]
         float* lsum = red + 2 * 2 * BM;                             // [2 halves][BM]
         const int lim = min(p.causal ? ctx - n + r0 + row : ctx - 1, ctx - 1);
+        const int row_lo = w > 0 ? max(0, ctx - n + r0 + row - w + 1) : 0;     // this row's first key
         const float sl2 = p.scale_log2;
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
@@ -346,10 +345,12 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
 #pragma unroll
             for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(r[c]);
             const int jt = tile_of(j);
-            if (jt * BN + BN - 1 > min_lim) {                       // diagonal / last tile: mask
+            if (jt * BN + BN - 1 > min_lim || jt * BN < lo_mask) {  // diagonal / last / window edge
 #pragma unroll
-                for (int c = 0; c < 64; ++c)
-                    if (jt * BN + c0 + c > lim) x[c] = -INFINITY;
+                for (int c = 0; c < 64; ++c) {
+                    const int key = jt * BN + c0 + c;
+                    if (key > lim || key < row_lo) x[c] = -INFINITY;
+                }
             }
             float mh = x[0];
 #pragma unroll
@@ -357,7 +358,8 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
             float* rb = red + (j & 1) * 2 * BM;
             rb[hf * BM + row] = mh;
             named_bar_sync(1 + quarter, 64);
-            const float mt = fmaxf(mh, rb[(1 - hf) * BM + row]) * sl2;   // finite: key 0 is visible
+            // -inf only for a row that sees no key of this tile (possible with a window)
+            const float mt = fmaxf(mh, rb[(1 - hf) * BM + row]) * sl2;
             if (j == 0) {
                 m_ref = mt;
             } else if (__any_sync(0xffffffffu, mt > m_ref + kRescaleThreshold)) {
@@ -385,7 +387,7 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
                 }
                 ptx::tc_wait_st();
             }
-            const float neg = -m_ref;
+            const float neg = m_ref == -INFINITY ? 0.f : -m_ref;      // no key seen yet: all p are 0
             float rs = 0.f;
 #pragma unroll
             for (int c16 = 0; c16 < 2; ++c16) {

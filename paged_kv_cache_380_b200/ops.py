@@ -26,6 +26,7 @@ _DT = {torch.float32: PKV_F32, torch.bfloat16: PKV_BF16, torch.float16: PKV_F16,
 # every symbol include/pagedkv.h declares
 EXPORTS = ("pkv_error_string", "pkv_kv_cache_write", "pkv_kv_cache_write_quant", "pkv_paged_attention_decode",
            "pkv_decode_workspace_size", "pkv_decode_plan", "pkv_paged_attention_decode_noalloc",
+           "pkv_paged_attention_decode_ex", "pkv_paged_attention_prefill_ex",
            "pkv_paged_attention_prefill",
            "pkv_get_device_status", "pkv_bm_create", "pkv_bm_destroy", "pkv_bm_add_sequence", "pkv_bm_fork",
            "pkv_bm_append", "pkv_bm_free_sequence", "pkv_bm_block_tables", "pkv_bm_num_free_pages",
@@ -58,6 +59,12 @@ def load(path: str = _LIB_PATH):
         lib.pkv_paged_attention_decode.argtypes = [P, P, P, P, P, F, P, I, I, I, I, I, I, I64, I, I,
                                                    P, P, P, SZ, I, P]
         lib.pkv_paged_attention_decode.restype = I
+        lib.pkv_paged_attention_decode_ex.argtypes = [P, P, P, P, P, F, P, I, I, I, I, I, I, I64, I, I,
+                                                      P, P, P, SZ, I, I, P]
+        lib.pkv_paged_attention_decode_ex.restype = I
+        lib.pkv_paged_attention_prefill_ex.argtypes = [P, P, P, P, P, P, I, F, P, I, I, I, I, I, I, I, I,
+                                                       I64, I, I, P]
+        lib.pkv_paged_attention_prefill_ex.restype = I
         lib.pkv_paged_attention_decode_noalloc.argtypes = [P, P, P, P, P, F, P, I, I, I, I, I, I, I64, I, I,
                                                            P, P, I, P]
         lib.pkv_paged_attention_decode_noalloc.restype = I
@@ -172,7 +179,7 @@ def decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, page_si
 
 
 def paged_attention_decode(q, k_pages, v_pages, block_tables, context_lens, scale, out=None, *,
-                           k_scales=None, v_scales=None, workspace=None, num_splits=0, stream=None):
+                           k_scales=None, v_scales=None, workspace=None, num_splits=0, window=0, stream=None):
     """Decode attention: ``q [B, Hq, D]`` against pools ``[P, ps, Hkv, D]``
     through ``block_tables int32 [B, MP]`` and ``context_lens int32 [B]``.
     Returns ``out`` (allocated like ``q`` if not given).  A workspace of
@@ -192,11 +199,14 @@ def paged_attention_decode(q, k_pages, v_pages, block_tables, context_lens, scal
     if workspace is None:
         need = decode_workspace_size(B, Hq, Hkv, D, ps, MP, kv_dt, num_splits)
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-    _check(load().pkv_paged_attention_decode(
-        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_tables), _ptr(context_lens), float(scale),
-        _ptr(out), B, Hq, Hkv, D, ps, MP, P, _dtype_code(q), _dtype_code(k_pages), _ptr(k_scales),
-        _ptr(v_scales), _ptr(workspace), workspace.numel(), int(num_splits), _stream(stream)),
-        "paged_attention_decode")
+    lib = load()
+    args = (_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_tables), _ptr(context_lens), float(scale),
+            _ptr(out), B, Hq, Hkv, D, ps, MP, P, _dtype_code(q), _dtype_code(k_pages), _ptr(k_scales),
+            _ptr(v_scales), _ptr(workspace), workspace.numel(), int(num_splits))
+    if window > 0:
+        _check(lib.pkv_paged_attention_decode_ex(*args, int(window), _stream(stream)), "paged_attention_decode_ex")
+    else:
+        _check(lib.pkv_paged_attention_decode(*args, _stream(stream)), "paged_attention_decode")
     return out
 
 
@@ -219,7 +229,7 @@ def paged_attention_decode_noalloc(q, k_pages, v_pages, block_tables, context_le
 
 
 def paged_attention_prefill(q, k_pages, v_pages, block_tables, q_start, context_lens, causal, scale,
-                            out=None, *, max_q_len=None, stream=None):
+                            out=None, *, max_q_len=None, window=0, stream=None):
     """Chunked prefill: packed ``q [Ttot, Hq, D]``, rows ``q_start[b]..q_start[b+1]-1``
     of sequence b at positions ``ctx-n..ctx-1``; causal rows see keys up to
     their own position.  ``max_q_len`` (the longest chunk) sizes the grid;
@@ -234,10 +244,14 @@ def paged_attention_prefill(q, k_pages, v_pages, block_tables, q_start, context_
         out = torch.empty_like(q)
     if max_q_len is None:
         max_q_len = int((q_start[1:] - q_start[:-1]).max().item()) if B else 0
-    _check(load().pkv_paged_attention_prefill(
-        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_tables), _ptr(q_start), _ptr(context_lens),
-        1 if causal else 0, float(scale), _ptr(out), B, T, int(max_q_len), Hq, Hkv, D, ps,
-        block_tables.shape[1], P, _dtype_code(q), _stream(stream)), "paged_attention_prefill")
+    lib = load()
+    args = (_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_tables), _ptr(q_start), _ptr(context_lens),
+            1 if causal else 0, float(scale), _ptr(out), B, T, int(max_q_len), Hq, Hkv, D, ps,
+            block_tables.shape[1], P, _dtype_code(q))
+    if window > 0:
+        _check(lib.pkv_paged_attention_prefill_ex(*args, int(window), _stream(stream)), "paged_attention_prefill_ex")
+    else:
+        _check(lib.pkv_paged_attention_prefill(*args, _stream(stream)), "paged_attention_prefill")
     return out
 
 

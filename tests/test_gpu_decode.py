@@ -15,7 +15,7 @@ pytestmark = pytest.mark.gpu
 TOL = {"bf16": 2e-2, "f16": 2e-2, "f32": 1e-4, "i8": 5e-2}
 
 
-def run_case(case, kv="same", num_splits=0, write_new=False, items=None):
+def run_case(case, kv="same", num_splits=0, write_new=False, items=None, window=0):
     """Run the GPU decode on a workloads.Case and compare with the oracle."""
     tag = case.dtype
     k_host, v_host = case.k_pages, case.v_pages
@@ -37,15 +37,15 @@ def run_case(case, kv="same", num_splits=0, write_new=False, items=None):
     q = dev(case.q, tag)
     bt, cl = dev(case.block_tables, "i32"), dev(case.context_lens, "i32")
     out = ops.paged_attention_decode(q, kp, vp, bt, cl, case.scale, k_scales=dks, v_scales=dvs,
-                                     num_splits=num_splits)
+                                     num_splits=num_splits, window=window)
     torch.cuda.synchronize()
     assert_status_ok()
     if kv == "i8":
         want = oracle.decode(case.q, tag, kq, vq, "i8", case.block_tables, case.context_lens, case.scale,
-                             k_scales=ks, v_scales=vs, items=items)
+                             k_scales=ks, v_scales=vs, items=items, window=window)
     else:
         want = oracle.decode(case.q, tag, k_host, v_host, tag, case.block_tables, case.context_lens,
-                             case.scale, items=items)
+                             case.scale, items=items, window=window)
     got = f64(out)
     if items is not None:
         got = got.reshape(-1, got.shape[-1])[items]
@@ -155,3 +155,17 @@ def test_int8_pages_large_queries():
     c.q = W.to_bf16_bits(q)
     c.scale = 1e-5
     run_case(c, kv="i8")
+
+
+# ---- local (sliding-window) attention ---------------------------------------------
+
+@pytest.mark.parametrize("window", [1, 16, 17, 100, 5000])
+@pytest.mark.parametrize("num_splits", [0, 3])
+def test_sliding_window_decode(window, num_splits):
+    run_case(small_case(90, Hq=8, Hkv=2, ctx=(1, 15, 16, 17, 33, 100, 0, 1000)), num_splits=num_splits,
+             window=window)
+
+
+def test_sliding_window_decode_int8_and_fp32():
+    run_case(small_case(91, Hq=8, Hkv=2, ctx=(5, 260, 1000)), kv="i8", window=70)
+    run_case(small_case(92, Hq=4, Hkv=2, D=64, dtype="f32", ctx=(1, 16, 0, 45)), window=9)

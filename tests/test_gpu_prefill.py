@@ -12,7 +12,7 @@ from paged_kv_cache_380_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 
 
-def run_prefill(case, causal=True, items=None, tol=2e-2):
+def run_prefill(case, causal=True, items=None, tol=2e-2, window=0):
     """Append the chunk's K/V (cache write), then prefill; compare with the oracle."""
     tag = case.dtype
     kp, vp = dev(case.k_pages, tag), dev(case.v_pages, tag)
@@ -22,11 +22,12 @@ def run_prefill(case, causal=True, items=None, tol=2e-2):
     q = dev(case.q, tag)
     max_q = int(np.max(np.diff(case.q_start))) if case.batch else 0
     out = ops.paged_attention_prefill(q, kp, vp, dev(case.block_tables, "i32"), dev(case.q_start, "i32"),
-                                      dev(case.context_lens, "i32"), causal, case.scale, max_q_len=max_q)
+                                      dev(case.context_lens, "i32"), causal, case.scale, max_q_len=max_q,
+                                      window=window)
     torch.cuda.synchronize()
     assert_status_ok()
     want = oracle.prefill(case.q, tag, k_host, v_host, tag, case.block_tables, case.q_start,
-                          case.context_lens, causal, case.scale, items=items)
+                          case.context_lens, causal, case.scale, items=items, window=window)
     got = f64(out)
     got = got.reshape(-1, got.shape[-1])[items] if items is not None else got
     assert_close(got, want, tol, case.name)
@@ -75,3 +76,14 @@ def test_chunked_prefill_shared_prefix_full():
     for t in (0, 1, 127, 128, 255, 511, 512, 1023, 2047, 4095):   # tile edges, sequence edges
         items |= {t * Hq + h for h in range(Hq)}
     run_prefill(c, items=np.array(sorted(items)))
+
+
+# ---- local (sliding-window) attention ---------------------------------------------
+
+@pytest.mark.parametrize("window", [1, 64, 128, 129, 300])
+def test_sliding_window_prefill(window):
+    run_prefill(case(20, chunks=(1, 5, 64, 130, 200, 128), private_prefix=7, shared_prefix=256), window=window)
+
+
+def test_sliding_window_prefill_non_causal():
+    run_prefill(case(21, chunks=(40, 129), private_prefix=3), causal=False, window=50)
