@@ -11,27 +11,30 @@
 // Flash Attention，让 Token 生成快 3 倍" ("Flash Attention 的分块计算原理"),
 // K/V read page by page through the block table.
 //
-// B200 design, one CTA per (128-row query tile, query head, sequence):
-//  * warp 0 = TMA producer: Q tile once (two 64-column SW128 boxes), then per
-//    128-key tile one 16-row box per page group and 64-column half for K and
-//    for V, into rings of 3 K stages and 2 V stages (mbarrier expect_tx).
-//  * warp 1 = MMA issuer (one thread): S_j = Q K_j^T (M=128, N=128, K=128,
-//    bf16 -> fp32 in TMEM, triple-buffered) and O += P_j V_j with P read from
-//    TMEM (the TS form) and V as an MN-major operand; tcgen05.commit signals
-//    S ready, the K stage free, O updated and the V stage free.
-//  * warps 2-9 = softmax: one TMEM lane (query row) per thread, two warps per
+// B200 design, one CTA per (128-row query tile, query head, sequence), 12 warps:
+//  * warps 0-2 = TMA producers: the Q tile once (two 64-column SW128 boxes), then
+//    per 128-key tile one 16-row box per page group and 64-column half for K and
+//    for V (lane pairs of the three warps split the 16 boxes of a tile), into
+//    rings of 3 K stages and 2 V stages (mbarrier expect_tx).
+//  * warp 3 = MMA issuer (one thread): S_j = Q K_j^T (M=128, N=128, K=128, bf16
+//    -> fp32 in TMEM, three S/P buffers) and O += P_j V_j with P read from TMEM
+//    (the TS form) and V as an MN-major operand.  S runs two tiles ahead of PV
+//    (S_0 S_1 | PV_0 S_2 | PV_1 S_3 ...), so the softmax of tile i+1 never waits
+//    for P_i.  One tcgen05.commit per MMA group (each commit costs tensor-pipe
+//    time): "S_j done" also frees K stage j, "PV_i done" also frees P buffer i
+//    and the V stage PV_i read.
+//  * warps 4-11 = softmax: one TMEM lane (query row) per thread, two warps per
 //    row quarter taking 64 columns each (row max and row sum exchanged in
 //    shared memory); tcgen05.ld of the S half-row, masking, max, 2^(s*scale -
-//    m) with the scale folded into one FFMA (one exponential in four on the
-//    FMA pipe as a polynomial, the rest on the SFU), row sum, P packed to bf16
-//    pairs and tcgen05.st back over the S columns.  The accumulator is rescaled only
-//    when a row's running max grows by more than 2^8 (P <= 256 otherwise),
-//    which keeps O's TMEM round trip off most tiles; the final division by
-//    the row sum makes any consistent reference max exact.
+//    m) with the scale folded into one FFMA, row sum, P packed to bf16 pairs
+//    and tcgen05.st back over the S columns; one P-ready arrival per warp.  The
+//    accumulator is rescaled only when a row's running max grows by more than
+//    2^8 (P <= 256 otherwise), which keeps O's TMEM round trip off most tiles;
+//    the final division by the row sum makes any consistent reference max exact.
 //  * Heaviest (longest causal) query tiles are launched first.
-//  * Every mbarrier wait is bounded; on time-out the CTA records
-//    PKV_ERR_DEVICE_TIMEOUT, raises an abort flag so every role leaves its
-//    loop, waits (bounded) for its own async work and frees TMEM.
+//  * Every mbarrier wait polls (test_wait) and is bounded in time; on time-out
+//    the CTA records PKV_ERR_DEVICE_TIMEOUT, raises an abort flag so every role
+//    leaves its loop, waits (bounded) for its own async work and frees TMEM.
 #include <cuda.h>
 
 #include <cmath>
@@ -60,10 +63,11 @@ constexpr int kSmemV = kSmemK + KST * kTile;
 constexpr int kSmemRed = kSmemV + VST * kTile;   // row-max / row-sum exchange between warp pairs
 constexpr int kRedBytes = (2 * 2 * BM + 2 * BM) * 4;
 constexpr int kSmemBar = kSmemRed + kRedBytes;
-constexpr int kNumBars = 1 + 2 * KST + 2 * VST + 3 * NSB + 1;
+constexpr int kNumBars = 1 + KST + VST + 3 * NSB + 1;
 constexpr int kSmemBytes = kSmemBar + kNumBars * 8 + 16 + 1024;   // + TMEM addr, abort flag, alignment
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kOCol = NSB * 128;           // O accumulator columns 384..511
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // bound of every mbarrier wait (1 s)
 constexpr float kRescaleThreshold = 8.0f;       // log2 units: rescale when the max grows by > 2^8
 #ifndef PKV_PREFILL_POLY_EVERY
 #define PKV_PREFILL_POLY_EVERY 0                 // 1 in N exponentials on the FMA pipe (0 = none)
@@ -105,30 +109,65 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int b_mn_major) {
            (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// mbarrier addresses, all in one array after the tiles.
+// mbarrier addresses, all in one array after the tiles.  Every tcgen05.commit costs
+// tensor-pipe time, so each MMA group signals exactly one barrier: s_done(b) =
+// "S in buffer b is ready and K stage b is free" (K stages and S buffers share
+// the ring index), pv_done(b) = "O is updated, P buffer b and the V stage that
+// PV read are free".
 struct Bars {
     uint32_t base;
     __device__ __forceinline__ uint32_t q_full() const { return base; }
     __device__ __forceinline__ uint32_t k_full(int i) const { return base + 8 * (1 + i); }
-    __device__ __forceinline__ uint32_t k_empty(int i) const { return base + 8 * (1 + KST + i); }
-    __device__ __forceinline__ uint32_t v_full(int i) const { return base + 8 * (1 + 2 * KST + i); }
-    __device__ __forceinline__ uint32_t v_empty(int i) const { return base + 8 * (1 + 2 * KST + VST + i); }
-    __device__ __forceinline__ uint32_t s_full(int i) const { return base + 8 * (1 + 2 * KST + 2 * VST + i); }
-    __device__ __forceinline__ uint32_t p_full(int i) const { return base + 8 * (1 + 2 * KST + 2 * VST + NSB + i); }
-    __device__ __forceinline__ uint32_t pv_done(int i) const { return base + 8 * (1 + 2 * KST + 2 * VST + 2 * NSB + i); }
-    __device__ __forceinline__ uint32_t mma_done() const { return base + 8 * (1 + 2 * KST + 2 * VST + 3 * NSB); }
+    __device__ __forceinline__ uint32_t v_full(int i) const { return base + 8 * (1 + KST + i); }
+    __device__ __forceinline__ uint32_t s_done(int i) const { return base + 8 * (1 + KST + VST + i); }
+    __device__ __forceinline__ uint32_t p_full(int i) const { return base + 8 * (1 + KST + VST + NSB + i); }
+    __device__ __forceinline__ uint32_t pv_done(int i) const { return base + 8 * (1 + KST + VST + 2 * NSB + i); }
+    __device__ __forceinline__ uint32_t mma_done() const { return base + 8 * (1 + KST + VST + 3 * NSB); }
 };
 
 // Bounded wait that also gives up as soon as another role raised the abort flag.
+// It polls with the non-blocking test_wait: the pipeline is latency-bound, and a
+// thread suspended inside try_wait resumes measurably later than a polling one
+// (13% of the prefill time on a 128-row causal workload).  The bound is 1 s of
+// %globaltimer, after which the CTA records PKV_ERR_DEVICE_TIMEOUT.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                          DeviceStatus* st) {
-    for (uint32_t i = 0; i < kSpinLimit; ++i) {
-        if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (ptx::mbar_test_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (;;) {
+        if (ptx::mbar_test_wait(bar, parity)) return true;
         if (*abort_flag) return false;
+        if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) break;
     }
     *abort_flag = 1;
     record_error(st, PKV_ERR_DEVICE_TIMEOUT, static_cast<long long>(bar));
     return false;
+}
+
+// One S tile: S[buffer SB] = Q K[stage SB]^T (K stages and S buffers share the index).
+template <typename T, int SB>
+__device__ __forceinline__ void mma_s(uint32_t sbase, const Bars& bars) {
+    static_assert(KST == NSB, "K stage and S buffer share one ring index");
+    constexpr uint32_t id_s = idesc_f16<T>(BM, BN, 0);
+    const uint32_t kbase = sbase + kSmemK + SB * kTile;
+#pragma unroll
+    for (int kk = 0; kk < HD / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
+        ptx::tc_mma_ss(SB * 128, sdesc(sbase + kSmemQ + off, 16, 1024), sdesc(kbase + off, 16, 1024), id_s,
+                       kk > 0 ? 1u : 0u);
+    }
+    ptx::tc_commit(bars.s_done(SB));
+}
+// One PV tile: O (+)= P[buffer PB] V[stage VS]; ACC = false only for the first tile.
+template <typename T, int PB, int VS, bool ACC>
+__device__ __forceinline__ void mma_pv(uint32_t sbase, const Bars& bars) {
+    constexpr uint32_t id_o = idesc_f16<T>(BM, HD, 1);
+    const uint32_t vbase = sbase + kSmemV + VS * kTile;
+#pragma unroll
+    for (int kk = 0; kk < BN / 16; ++kk)
+        ptx::tc_mma_ts(kOCol, PB * 128 + kk * 8, sdesc(vbase + kk * 2048, kAtom, 1024), id_o,
+                       (ACC || kk > 0) ? 1u : 0u);
+    ptx::tc_commit(bars.pv_done(PB));
 }
 
 template <typename T>
@@ -183,17 +222,11 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
 
     if (threadIdx.x == 0) {
         ptx::mbar_init(bars.q_full(), 1);
-        for (int i = 0; i < KST; ++i) {
-            ptx::mbar_init(bars.k_full(i), kProducerWarps);
-            ptx::mbar_init(bars.k_empty(i), 1);
-        }
-        for (int i = 0; i < VST; ++i) {
-            ptx::mbar_init(bars.v_full(i), kProducerWarps);
-            ptx::mbar_init(bars.v_empty(i), 1);
-        }
+        for (int i = 0; i < KST; ++i) ptx::mbar_init(bars.k_full(i), kProducerWarps);
+        for (int i = 0; i < VST; ++i) ptx::mbar_init(bars.v_full(i), kProducerWarps);
         for (int i = 0; i < NSB; ++i) {
-            ptx::mbar_init(bars.s_full(i), 1);
-            ptx::mbar_init(bars.p_full(i), kSoftmaxWarps * 32);
+            ptx::mbar_init(bars.s_done(i), 1);
+            ptx::mbar_init(bars.p_full(i), kSoftmaxWarps);
             ptx::mbar_init(bars.pv_done(i), 1);
         }
         ptx::mbar_init(bars.mma_done(), 1);
@@ -207,7 +240,13 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
+    // All 512 columns are allocated, so the allocation starts at lane 0, column 0
+    // and the MMAs use constant TMEM addresses; anything else is reported.
+    const uint32_t tmem = 0;
+    if (threadIdx.x == 0 && *tmem_slot != 0u) {
+        *abort_flag = 1;
+        record_error(p.status, PKV_ERR_CUDA, static_cast<long long>(*tmem_slot));
+    }
 
     if (warp < kProducerWarps) {
         // ------------------------------ TMA producers ------------------------------
@@ -243,8 +282,13 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
             const int nst = is_k ? KST : VST, st = t % nst;
             const unsigned nbox = __popc(__ballot_sync(0xffffffffu, row >= 0));
             bool ok = true;
-            if (t >= nst)
-                ok = wait_bar(is_k ? bars.k_empty(st) : bars.v_empty(st), ((t / nst) - 1) & 1, abort_flag, p.status);
+            // a K stage is free once S of the tile KST back is done, a V stage once
+            // PV of the tile VST back is done
+            if (t >= nst) {
+                const int prev = t - nst;
+                ok = wait_bar(is_k ? bars.s_done(prev % NSB) : bars.pv_done(prev % NSB), (prev / NSB) & 1,
+                              abort_flag, p.status);
+            }
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             if (!ok) return false;
             const uint32_t bar = is_k ? bars.k_full(st) : bars.v_full(st);
@@ -272,42 +316,44 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------ MMA issuer ------------------------------
+        // S runs two tiles ahead of PV (S_0 S_1 | PV_0 S_2 | PV_1 S_3 | ...), so the
+        // softmax of tile i+1 never waits for P_i.  The ring slots are template
+        // arguments of the issue helpers and the TMEM base is 0, so every MMA
+        // operand is a constant.
         if (lane == 0) {
-            constexpr uint32_t id_s = idesc_f16<T>(BM, BN, 0);
-            constexpr uint32_t id_o = idesc_f16<T>(BM, HD, 1);
             bool ok = wait_bar(bars.q_full(), 0, abort_flag, p.status);
-            auto issue_pv = [&](int i) {
-                const int bi = i % NSB, vs = i % VST;
-                if (!wait_bar(bars.p_full(bi), (i / NSB) & 1, abort_flag, p.status)) return false;
-                if (!wait_bar(bars.v_full(vs), (i / VST) & 1, abort_flag, p.status)) return false;
+            auto issue_s = [&](int j) {
+                if (!wait_bar(bars.k_full(j % KST), (j / KST) & 1, abort_flag, p.status)) return false;
+                if (j >= NSB && !wait_bar(bars.pv_done(j % NSB), ((j / NSB) - 1) & 1, abort_flag, p.status))
+                    return false;
                 ptx::tc_fence_after();
-                const uint32_t vbase = sbase + kSmemV + vs * kTile;
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk)
-                    ptx::tc_mma_ts(tmem + kOCol, tmem + bi * 128 + kk * 8,
-                                   sdesc(vbase + kk * 2048, kAtom, 1024), id_o, (i > 0 || kk > 0) ? 1u : 0u);
-                ptx::tc_commit(bars.pv_done(bi));
-                ptx::tc_commit(bars.v_empty(vs));
+                switch (j % 3) {
+                    case 0: mma_s<T, 0>(sbase, bars); break;
+                    case 1: mma_s<T, 1>(sbase, bars); break;
+                    default: mma_s<T, 2>(sbase, bars); break;
+                }
                 return true;
             };
-            for (int j = 0; j < n_tiles && ok; ++j) {
-                const int ks = j % KST, bj = j % NSB;
-                ok = wait_bar(bars.k_full(ks), (j / KST) & 1, abort_flag, p.status);
-                if (ok && j >= NSB) ok = wait_bar(bars.pv_done(bj), ((j / NSB) - 1) & 1, abort_flag, p.status);
-                if (!ok) break;
+            auto issue_pv = [&](int i) {
+                if (!wait_bar(bars.p_full(i % NSB), (i / NSB) & 1, abort_flag, p.status)) return false;
+                if (!wait_bar(bars.v_full(i % VST), (i / VST) & 1, abort_flag, p.status)) return false;
                 ptx::tc_fence_after();
-                const uint32_t kbase = sbase + kSmemK + ks * kTile;
-#pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
-                    ptx::tc_mma_ss(tmem + bj * 128, sdesc(sbase + kSmemQ + off, 16, 1024),
-                                   sdesc(kbase + off, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+                switch (i == 0 ? -1 : i % 6) {
+                    case -1: mma_pv<T, 0, 0, false>(sbase, bars); break;
+                    case 0: mma_pv<T, 0, 0, true>(sbase, bars); break;
+                    case 1: mma_pv<T, 1, 1, true>(sbase, bars); break;
+                    case 2: mma_pv<T, 2, 0, true>(sbase, bars); break;
+                    case 3: mma_pv<T, 0, 1, true>(sbase, bars); break;
+                    case 4: mma_pv<T, 1, 0, true>(sbase, bars); break;
+                    default: mma_pv<T, 2, 1, true>(sbase, bars); break;
                 }
-                ptx::tc_commit(bars.s_full(bj));
-                ptx::tc_commit(bars.k_empty(ks));
-                if (j >= 1) ok = issue_pv(j - 1);
+                return true;
+            };
+            ok = ok && issue_s(0) && (n_tiles < 2 || issue_s(1));
+            for (int i = 0; i < n_tiles && ok; ++i) {
+                ok = issue_pv(i);
+                if (ok && i + 2 < n_tiles) ok = issue_s(i + 2);
             }
-            if (ok) issue_pv(n_tiles - 1);
             // drain: every tcgen05 op issued by this thread completes before TMEM is freed
             ptx::tc_commit(bars.mma_done());
             ptx::mbar_wait(bars.mma_done(), 0, kSpinLimit);
@@ -330,7 +376,7 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
         bool ok = true;
         for (int j = 0; j < n_tiles; ++j) {
             const int bj = j % NSB;
-            ok = wait_bar(bars.s_full(bj), (j / NSB) & 1, abort_flag, p.status);
+            ok = wait_bar(bars.s_done(bj), (j / NSB) & 1, abort_flag, p.status);
             if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
             ptx::tc_fence_after();
             uint32_t r[64];
@@ -421,7 +467,8 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
                 ptx::fence_proxy_async_smem();
             }
             ptx::tc_fence_before();
-            ptx::mbar_arrive(bars.p_full(bj));
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bars.p_full(bj));      // one arrival per warp
         }
         // epilogue: O / l -> out (each warp writes its 64 output columns)
         if (ok) {
@@ -461,7 +508,7 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
     }
     if (warp == kMmaWarp) {
         ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem, kTmemCols);
+        ptx::tmem_dealloc(*tmem_slot, kTmemCols);
     }
 }
 
@@ -507,9 +554,9 @@ cudaError_t run(const PrefillParams& p, cudaStream_t stream) {
         !make_map(&tk, p.k_pages, dt, p.num_kv_heads, pool_rows, 16) ||
         !make_map(&tv, p.v_pages, dt, p.num_kv_heads, pool_rows, 16))
         return cudaErrorInvalidValue;
+    dim3 grid(p.num_q_heads, p.num_seqs, ceil_div(p.max_q_len, BM));
     cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(prefill_tc_kernel<T>), kSmemBytes);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.num_q_heads, p.num_seqs, ceil_div(p.max_q_len, BM));
     prefill_tc_kernel<T><<<grid, kThreads, kSmemBytes, stream>>>(p, tq, tk, tv);
     return cudaGetLastError();
 }
