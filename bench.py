@@ -53,7 +53,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic per launch of the dominant kernel from an ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by workload, with the
 # hash of the kernel sources it was taken on; reported only while they match.
-TRAFFIC = {}
+TRAFFIC = {
+    # decode_mma_kernel: 585.82 MB per launch at batch 16 (the capture-size case), 1.0075 x its
+    # algorithmic bytes; scaled to the batch-64 launch by algorithmic bytes (2346.49 MB)
+    "llama2_7b_mha_decode": {"bytes": 2363970000, "kernel_sha": "b47d14b81414f9e0"},
+    # prefill_tc_kernel: 54.66 MB read + 4.87 MB written per launch, full workload, cold L2
+    "chunked_prefill_shared_prefix": {"bytes": 59527936, "kernel_sha": "bf153121dbf992a1"},
+}
 KERNEL_SOURCES = {
     "decode": ["paged_kv_cache_380_b200/csrc/decode.cu", "paged_kv_cache_380_b200/csrc/pkv_ptx.cuh",
                "paged_kv_cache_380_b200/csrc/pkv_common.cuh"],

@@ -69,24 +69,6 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kOCol = NSB * 128;           // O accumulator columns 384..511
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // bound of every mbarrier wait (1 s)
 constexpr float kRescaleThreshold = 8.0f;       // log2 units: rescale when the max grows by > 2^8
-#ifndef PKV_PREFILL_POLY_EVERY
-#define PKV_PREFILL_POLY_EVERY 0                 // 1 in N exponentials on the FMA pipe (0 = none)
-#endif
-constexpr int kPolyEvery = PKV_PREFILL_POLY_EVERY;
-
-// 2^x on the FMA/ALU pipes, for softmax arguments x <= 8: Cody-Waite split
-// x = n + f with n = round(x) (the 1.5 * 2^23 shifter), f in [-0.5, 0.5];
-// 2^f from a degree-3 polynomial fitted here for least relative error on
-// [-0.5, 0.5] (iteratively reweighted least squares, max relative error
-// 7.5e-5, below the bf16 rounding P gets anyway); 2^n added into the
-// exponent field.  Arguments below -126 are clamped (result ~1e-38 instead of 0).
-__device__ __forceinline__ float exp2_poly(float x) {
-    x = fmaxf(x, -126.0f);
-    const float t = x + 12582912.0f;
-    const float f = x - (t - 12582912.0f);
-    const float q = fmaf(fmaf(fmaf(0.055166300f, f, 0.24261182f), f, 0.69326228f), f, 0.99992806f);
-    return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
-}
 
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");
@@ -442,8 +424,7 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
                 for (int i = 0; i < 16; ++i) {
                     const int c = c16 * 32 + 2 * i;
                     const float ya = fmaf(x[c], sl2, neg), yb = fmaf(x[c + 1], sl2, neg);
-                    const float a = (kPolyEvery && (c % kPolyEvery) == kPolyEvery - 1) ? exp2_poly(ya) : ptx::ex2(ya);
-                    const float bb = (kPolyEvery && ((c + 1) % kPolyEvery) == kPolyEvery - 1) ? exp2_poly(yb) : ptx::ex2(yb);
+                    const float a = ptx::ex2(ya), bb = ptx::ex2(yb);
                     rs += a + bb;
                     pk[i] = pack2<T>(a, bb);
                 }
