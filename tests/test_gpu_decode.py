@@ -83,6 +83,12 @@ def test_page_sizes_and_head_dims(ps, D):
     run_case(small_case(ps + D, Hq=8, Hkv=2, D=D, ps=ps, ctx=(1, 31, 32, 257, 600)), num_splits=2)
 
 
+@pytest.mark.parametrize("num_splits", [0, 2])
+def test_partition_boundaries(num_splits):
+    # contexts on either side of the 1024-token split partitions and of whole pages
+    run_case(small_case(9, Hq=16, Hkv=4, ctx=(1023, 1024, 1025, 2047, 2048, 2049, 4096, 1)), num_splits=num_splits)
+
+
 def test_fp16_pages():
     run_case(small_case(50, Hq=16, Hkv=4, dtype="f16"), num_splits=2)
 

@@ -87,3 +87,23 @@ def test_sliding_window_prefill(window):
 
 def test_sliding_window_prefill_non_causal():
     run_prefill(case(21, chunks=(40, 129), private_prefix=3), causal=False, window=50)
+
+
+# ---- more page sizes, GQA groups and batch shapes ----------------------------------
+
+@pytest.mark.parametrize("ps", [32, 64])
+def test_mid_size_pages(ps):
+    # 2 or 4 sixteen-row TMA page groups per page; chunks start mid-page
+    run_prefill(case(7 + ps // 32, chunks=(1, 31, 129, 200), private_prefix=5, shared_prefix=64, ps=ps))
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(16, 2), (16, 1)])
+def test_large_gqa_groups(Hq, Hkv):
+    # 8 and 16 query heads read the same KV head
+    run_prefill(case(10 + Hkv, chunks=(77, 130), Hq=Hq, Hkv=Hkv, private_prefix=9))
+
+
+def test_many_ragged_sequences():
+    # 40 sequences, seeded chunk lengths 0..149 (some empty), one shared prefix
+    chunks = np.random.default_rng(7).integers(0, 150, 40)
+    run_prefill(case(13, chunks=tuple(int(c) for c in chunks), private_prefix=3, shared_prefix=48))
