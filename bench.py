@@ -7,10 +7,12 @@ step: the cache append of the 64 new K/V rows (random slot mapping) followed
 by decode attention of 64 sequences (32/32 heads, head_dim 128, bf16, page
 16, contexts uniform in [512, 4096]), split-KV partitions and their merge
 included.  ``--workload`` selects the other workloads (GQA decode, long
-context bf16/INT8, chunked prefill with a shared prefix, tiny fp32 decode).
+context bf16/INT8, chunked prefill with a shared prefix, tiny fp32 decode), and
+``kv_cache_write_full`` the cache append at bandwidth scale (every cached token of
+the Llama-2-7B-shaped batch written through a random slot permutation).
 
 Prints ONE JSON line (rank 0).  ``value`` is whole-job throughput: algorithmic
-bytes (decode) or flops (prefill) of all ranks' steps divided by the device
+bytes (decode, cache append) or flops (prefill) of all ranks' steps divided by the device
 time of the timed steps (CUDA events on the launching stream, max over ranks).
 ``e2e`` repeats the measurement through the public API from pinned host
 buffers, with the per-step host->device copies of the step's inputs and the
@@ -342,8 +344,61 @@ class PrefillStep:
                 "l2": "L2 flushed between steps (252 MB write outside the events)"}
 
 
+class ScatterStep:
+    """The cache append at bandwidth scale: every cached token of the Llama-2-7B-shaped
+    decode batch (143 k rows of K and of V, 8 KiB each) is written again through a
+    seeded random permutation of the pool's slots.  Bytes per step: the K and V rows
+    read and written, plus the slots."""
+
+    kind = "scatter"
+
+    def __init__(self, case):
+        import torch
+        from paged_kv_cache_380_b200 import workloads as W
+        self.case = case
+        tag = case.dtype
+        self.src, self.dst = W.full_cache_scatter(case)
+        self.kp, self.vp = dev(case.k_pages, tag), dev(case.v_pages, tag)
+        Hkv, D = case.num_kv_heads, case.head_dim
+        src = torch.as_tensor(self.src, device="cuda")
+        self.k_new = self.kp.view(-1, Hkv, D)[src].clone()     # the cached rows, in sequence order
+        self.v_new = self.vp.view(-1, Hkv, D)[src].clone()
+        self.slots = dev(self.dst, "i64")
+        T = int(self.src.shape[0])
+        self.row_bytes = Hkv * D * self.kp.element_size()
+        self.work = 2 * 2 * T * self.row_bytes + 8 * T          # bytes per step
+        self.units = T
+        self.launches = 1
+        # the step's result read back end to end: the first destination row of K
+        self.out = self.kp.view(-1, Hkv * D)[int(self.dst[0])]
+
+    def run(self, ev=None):
+        from paged_kv_cache_380_b200 import ops
+        if ev is not None:
+            ev[0].record()
+        ops.kv_cache_write(self.k_new, self.v_new, self.slots, self.kp, self.vp)
+        if ev is not None:
+            ev[1].record()
+
+    def host_io(self):
+        import torch
+        ins = [self.k_new, self.v_new, self.slots]
+        hosts = [t.cpu().pin_memory() for t in ins]
+        out_h = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        return list(zip(hosts, ins)), out_h
+
+    def config(self):
+        c = self.case
+        return {"workload": "kv_cache_write_full", "rows": self.units, "row_bytes": self.row_bytes,
+                "num_kv_heads": c.num_kv_heads, "head_dim": c.head_dim, "page_size": c.page_size,
+                "slots": "seeded random permutation of the pool's slots",
+                "l2": "inputs and pool rows (4.7 GB) far above L2"}
+
+
 def make_step(name: str, batch: int = 0, graph: bool = False, window: int = 0):
     from paged_kv_cache_380_b200 import workloads as W
+    if name == "kv_cache_write_full":
+        return ScatterStep(W.llama2_7b_mha_decode(**({"batch": batch} if batch else {})))
     if name == "long_ctx_split_kv_int8":
         step = DecodeStep(W.long_ctx_split_kv(**({"batch": batch} if batch else {})), int8=True, window=window)
         return GraphStep(step) if graph else step
@@ -422,11 +477,30 @@ def time_e2e(step, K):
     return sum(s.elapsed_time(e) for s, e in zip(starts, ends)), h2d, d2h
 
 
+def _oracle_scatter_rate(case, src, dst, n_rows):
+    """The oracle's row copy of the first n_rows of a full-cache scatter into host copies of
+    the pools; returns (bytes per second, seconds)."""
+    import oracle
+    Hkv, D = case.num_kv_heads, case.head_dim
+    k_rows = case.k_pages.reshape(-1, Hkv, D)[src[:n_rows]]
+    v_rows = case.v_pages.reshape(-1, Hkv, D)[src[:n_rows]]
+    kp, vp = case.k_pages.copy(), case.v_pages.copy()
+    t0 = time.perf_counter()
+    oracle.kv_cache_write(k_rows, v_rows, dst[:n_rows], kp, vp)
+    dt = max(time.perf_counter() - t0, 1e-9)
+    return (2 * 2 * n_rows * k_rows[0].nbytes + 8 * n_rows) / dt, dt
+
+
 def cpu_baseline(step, budget_s: float = 20.0):
     """The fp64 oracle on the host cores over a bounded sample of the workload."""
     import oracle
     c = step.case
     threads = oracle.max_threads()
+    if step.kind == "scatter":
+        T = step.units
+        rate, dt = _oracle_scatter_rate(c, step.src, step.dst, T)
+        return {"value": rate / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                "sample": f"all {T} rows of the scatter, one row copy each ({dt:.2f} s)", "seconds": dt}
     if step.kind == "decode":
         B = c.batch
         # sample: the first S sequences (all heads), S sized to ~budget from a 1-sequence probe
@@ -532,12 +606,13 @@ def run_ours(args):
         raise RuntimeError(f"device status after timing: {ops.error_string(code)} ({detail})")
 
     peaks, peak_src = load_peaks()
-    scale_div = 1e9 if step.kind == "decode" else 1e12
-    unit = "GB/s" if step.kind == "decode" else "TFLOP/s"
+    hbm = step.kind in ("decode", "scatter")
+    scale_div = 1e9 if hbm else 1e12
+    unit = "GB/s" if hbm else "TFLOP/s"
     value = work / (elapsed / 1e3) / scale_div
     dom_avg_ms = statistics.mean(dom_ms)
-    if step.kind == "decode":
-        dom_work = step.decode_bytes
+    if hbm:
+        dom_work = step.decode_bytes if step.kind == "decode" else step.work
         peak = peaks["hbm_gbs"]
         achieved = dom_work / (dom_avg_ms / 1e3) / 1e9
         bound, runit = "hbm", "GB/s"
@@ -551,17 +626,21 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": round(elapsed / K, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "i8" if getattr(step, "int8", False) else step.case.dtype,
+        "vs_baseline": None, "dtype": ("u8" if step.kind == "scatter" else "i8" if getattr(step, "int8", False)
+                  else step.case.dtype),
         "data": "synthetic (seeded N(0,1) inputs, shuffled physical pages)",
         "config": dict(step.config(), parallelism=f"replicas{world}" if world > 1 else "single-gpu"),
         "impl": "ours",
         "extra": ({"tokens_per_s": round(units / (elapsed / 1e3), 1),
                    "pct_of_8TBps": round(100 * value / 8000.0, 2)} if step.kind == "decode"
+                  else {"rows_per_s": round(units / (elapsed / 1e3), 1),
+                        "pct_of_8TBps": round(100 * value / 8000.0, 2)} if step.kind == "scatter"
                   else {"rows_per_s": round(units / (elapsed / 1e3), 1)}),
         "roofline": {"bound": bound, "achieved": round(achieved, 3), "peak": peak, "unit": runit,
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "kernel": ("graph replay (append + decode + merge)" if args.graph else
                                 "decode call (main kernel + split-KV merge)" if step.kind == "decode"
+                                else "cache append (scatter kernel)" if step.kind == "scatter"
                                 else "prefill kernel"),
                      "kernel_ms": round(dom_avg_ms, 5), "peak_source": f"{peak_src} (MEASURED_PEAKS.json)"
                      if peak_src == "measured" else "fallback"},
@@ -590,6 +669,28 @@ def run_reference(args):
     import oracle
     from paged_kv_cache_380_b200 import workloads as W
     name = args.workload
+    if name == "kv_cache_write_full":
+        case = W.llama2_7b_mha_decode()
+        src, dst = W.full_cache_scatter(case)
+        Wm, K = max(3, args.warmup), args.steps
+        for _ in range(Wm):
+            _oracle_scatter_rate(case, src, dst, src.shape[0])
+        total = 0.0
+        nbytes = 2 * 2 * int(src.shape[0]) * case.num_kv_heads * case.head_dim * 2 + 8 * int(src.shape[0])
+        for _ in range(K):
+            total += _oracle_scatter_rate(case, src, dst, src.shape[0])[1]
+        value = nbytes * K / total / 1e9
+        sample = f"all {src.shape[0]} rows per step (row copies into host copies of the pools)"
+        print(json.dumps({"metric": METRIC, "value": round(value, 6), "unit": "GB/s", "n_gpus": world, "steps": K,
+                          "warmup": Wm, "ms_per_step": round(total / K * 1e3, 3), "higher_is_better": True,
+                          "scaling": "weak", "vs_baseline": None, "dtype": "u8",
+                          "data": "synthetic (seeded N(0,1) inputs, shuffled physical pages)",
+                          "config": {"workload": name, "parallelism": "host cores"}, "impl": "reference",
+                          "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": oracle.max_threads(),
+                                           "kind": "oracle", "sample": sample},
+                          "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}), flush=True)
+        return
     int8 = name == "long_ctx_split_kv_int8"
     case = W.long_ctx_split_kv() if int8 else W.WORKLOADS[name]()
 
@@ -645,11 +746,13 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama2_7b_mha_decode",
                     choices=["tiny_decode_f32", "llama2_7b_mha_decode", "llama2_70b_gqa_decode",
-                             "long_ctx_split_kv", "long_ctx_split_kv_int8", "chunked_prefill_shared_prefix"])
+                             "long_ctx_split_kv", "long_ctx_split_kv_int8", "chunked_prefill_shared_prefix",
+                             "kv_cache_write_full"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph", action="store_true",
                     help="decode workloads: replay the step as one captured CUDA graph")
-    ap.add_argument("--batch", type=int, default=0, help="override the batch size of a decode workload")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the batch size of a decode workload (or of kv_cache_write_full's source batch)")
     ap.add_argument("--window", type=int, default=0, help="local attention: attend only the last W keys")
     ap.add_argument("--cpu-seconds", type=float, default=20.0, help="CPU-baseline sample budget")
     ap.add_argument("--ref-seqs", type=int, default=4, help="reference arm: sequences per step (decode)")

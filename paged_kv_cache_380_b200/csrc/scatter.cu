@@ -8,8 +8,9 @@
 // so it is bit-exact for every dtype.
 //
 // HBM-bound: every thread moves U vectors of VEC bytes, issuing all U loads
-// before the U stores so each SM keeps tens of KB in flight; the grid is a
-// multiple of the SM count and grid-strides over (tensor, token, vector).
+// before the U stores so each SM keeps tens of KB in flight; the grid is the
+// number of CTAs that can be resident at once (one wave: a partial second wave
+// cost a quarter of the bandwidth) and grid-strides over (tensor, token, vector).
 #include "pkv_kernels.h"
 
 namespace pkv {
@@ -132,6 +133,15 @@ kv_quant_scatter_kernel(const T* __restrict__ src_k, const T* __restrict__ src_v
     }
 }
 
+// CTAs of `kernel` (256 threads, no dynamic shared memory) resident on the whole GPU.
+template <typename K>
+unsigned resident_ctas(K kernel) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
+    return static_cast<unsigned>(per_sm * sm_count());
+}
+
 }  // namespace
 
 cudaError_t launch_kv_quant_scatter(const void* src_k, const void* src_v, pkv_dtype src_dtype,
@@ -141,7 +151,7 @@ cudaError_t launch_kv_quant_scatter(const void* src_k, const void* src_v, pkv_dt
     if (num_tokens == 0) return cudaSuccess;
     const uint64_t rows = static_cast<uint64_t>(num_tokens) * num_kv_heads * 2;
     const uint64_t want = (rows + 7) / 8;
-    const uint64_t cap = static_cast<uint64_t>(sm_count()) * 16;
+    static const unsigned cap = resident_ctas(kv_quant_scatter_kernel<__nv_bfloat16, 4>);
     const unsigned blocks = static_cast<unsigned>(want < cap ? want : cap);
     auto* kp = static_cast<int8_t*>(k_pages);
     auto* vp = static_cast<int8_t*>(v_pages);
@@ -176,8 +186,11 @@ cudaError_t launch_kv_scatter(const void* src_k, const void* src_v, const int64_
     const uint64_t row_vecs = static_cast<uint64_t>(row_bytes) / vec;
     const uint64_t total = 2 * static_cast<uint64_t>(num_tokens) * row_vecs;
     const uint64_t want = (total + kThreads * kUnroll - 1) / (kThreads * kUnroll);
-    const uint64_t cap = static_cast<uint64_t>(sm_count()) * 8;
-    const unsigned blocks = static_cast<unsigned>(want < cap ? want : cap);
+    static const unsigned cap[5] = {resident_ctas(kv_scatter_kernel<1>), resident_ctas(kv_scatter_kernel<2>),
+                                    resident_ctas(kv_scatter_kernel<4>), resident_ctas(kv_scatter_kernel<8>),
+                                    resident_ctas(kv_scatter_kernel<16>)};
+    const unsigned c = cap[vec == 16 ? 4 : vec == 8 ? 3 : vec == 4 ? 2 : vec == 2 ? 1 : 0];
+    const unsigned blocks = static_cast<unsigned>(want < c ? want : c);
     const auto* sk = static_cast<const uint8_t*>(src_k);
     const auto* sv = static_cast<const uint8_t*>(src_v);
     auto* dk = static_cast<uint8_t*>(dst_k);

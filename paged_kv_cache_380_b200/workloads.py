@@ -316,6 +316,32 @@ def chunked_prefill_shared_prefix(num_seqs: int = 8, prefix: int = 1024, chunk: 
                         shared_prefix=prefix, chunk_lens=np.full(num_seqs, chunk))
 
 
+def cached_token_slots(case: Case) -> np.ndarray:
+    """Pool slot of every cached token of a decode case, sequence by sequence (int64)."""
+    ps = case.page_size
+    out = []
+    for b in range(case.batch):
+        n = int(case.context_lens[b])
+        pos = np.arange(n, dtype=np.int64)
+        pages = case.block_tables[b, :(n + ps - 1) // ps].astype(np.int64)
+        out.append(pages[pos // ps] * ps + pos % ps)
+    return np.concatenate(out) if out else np.zeros(0, np.int64)
+
+
+def full_cache_scatter(case: Case):
+    """The bandwidth case of the cache append: every cached token of ``case`` is
+    written again, to a seeded random permutation of the pool's slots.
+
+    Returns (src_slots, dst_slots): row t of the scatter is pool row src_slots[t]
+    (its K and V values), written to slot dst_slots[t] (distinct slots).
+    """
+    src = cached_token_slots(case)
+    num_slots = case.k_pages.shape[0] * case.page_size
+    rng = np.random.default_rng(np.random.SeedSequence(380 + case.meta["config_index"]).spawn(7)[6])
+    dst = rng.permutation(num_slots)[: src.shape[0]].astype(np.int64)
+    return src, dst
+
+
 WORKLOADS = {
     "tiny_decode_f32": tiny_decode_f32,
     "llama2_7b_mha_decode": llama2_7b_mha_decode,

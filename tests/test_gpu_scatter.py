@@ -68,6 +68,17 @@ def test_scatter_llama2_7b_new_tokens_bit_exact():
     _check_scatter(c.k_new, c.v_new, c.slot_mapping, c.k_pages, c.v_pages, "bf16")
 
 
+def test_scatter_full_cache_bit_exact():
+    """The bandwidth case bench.py times: all 143 k cached rows of the Llama-2-7B-shaped
+    batch written through a seeded random permutation of the pool's slots."""
+    c = W.llama2_7b_mha_decode()
+    src, dst = W.full_cache_scatter(c)
+    Hkv, D = c.num_kv_heads, c.head_dim
+    k_rows = c.k_pages.reshape(-1, Hkv, D)[src]
+    v_rows = c.v_pages.reshape(-1, Hkv, D)[src]
+    _check_scatter(k_rows, v_rows, dst, c.k_pages, c.v_pages, "bf16")
+
+
 def test_scatter_prefill_chunk_bit_exact():
     c = W.chunked_prefill_shared_prefix()
     _check_scatter(c.k_new, c.v_new, c.slot_mapping, c.k_pages, c.v_pages, "bf16")

@@ -68,3 +68,18 @@ def test_decode_append_slots_point_at_last_position():
         assert c.slot_mapping[b] == p * 4 + (ctx - 1) % 4
         flat = c.k_pages.reshape(-1, 1, 8)
         assert (flat[c.slot_mapping[b]] == W.CANARY_BITS["bf16"]).all()   # not yet written
+
+
+def test_full_cache_scatter_covers_every_cached_token_once():
+    c = W.decode_case(name="fc", config_index=77, batch=5, num_q_heads=4, num_kv_heads=2, head_dim=64,
+                      page_size=16, dtype="bf16", context_lens=np.array([0, 1, 16, 17, 100]))
+    src, dst = W.full_cache_scatter(c)
+    # brute force over the block tables: sequence by sequence, position by position
+    want = [int(c.block_tables[b, i // 16]) * 16 + i % 16
+            for b in range(c.batch) for i in range(int(c.context_lens[b]))]
+    assert src.tolist() == want
+    n_slots = c.k_pages.shape[0] * 16
+    assert dst.shape == src.shape and len(set(dst.tolist())) == dst.shape[0]
+    assert dst.min() >= 0 and dst.max() < n_slots
+    src2, dst2 = W.full_cache_scatter(c)                  # seeded: same draw every time
+    assert (src2 == src).all() and (dst2 == dst).all()
