@@ -302,7 +302,8 @@ int pkv_paged_attention_prefill_ex(const void* q, const void* k_pages, const voi
         return PKV_ERR_INVALID_ARG;
     if (dtype != PKV_BF16 && dtype != PKV_F16) return PKV_ERR_UNSUPPORTED;
     if (head_dim != 128 || page_size % kChunk) return PKV_ERR_UNSUPPORTED;
-    if (!aligned(q, 16) || !aligned(out, 4) || !aligned(k_pages, 16) || !aligned(v_pages, 16))
+    // q and the pools are TMA tensor-map bases; out is written with 16-byte stores
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16))
         return PKV_ERR_INVALID_ARG;
     DeviceStatus* st = status_ptr();
     if (!st) return PKV_ERR_CUDA;

@@ -105,6 +105,10 @@ def test_host_validation_rejects_before_launch(lib):
     rc = lib.pkv_paged_attention_prefill(fake, fake, fake, fake, fake, fake, 1, 1.0, fake, 2, 8, 4, 8, 2,
                                          128, 16, 4, 10, 0, None)
     assert rc == -2
+    # prefill output written with 16-byte stores: a 4-byte-aligned out is refused up front
+    rc = lib.pkv_paged_attention_prefill(fake, fake, fake, fake, fake, fake, 1, 1.0, P(0x10004), 2, 8, 4, 8, 2,
+                                         128, 16, 4, 10, 1, None)
+    assert rc == -1
     # empty problems are no-ops
     assert lib.pkv_paged_attention_decode(None, None, None, None, None, 1.0, None, 0, 8, 2, 128, 16, 4,
                                           10, 1, 1, None, None, None, 0, 0, None) == 0
