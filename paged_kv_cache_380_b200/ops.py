@@ -122,6 +122,15 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
+def _out_like(q, out):
+    """The output tensor: a new one like q, or the caller's, which must match q."""
+    if out is None:
+        return torch.empty_like(q)
+    if out.shape != q.shape or out.dtype != q.dtype:
+        raise ValueError(f"out must match q: got {tuple(out.shape)} {out.dtype}, want {tuple(q.shape)} {q.dtype}")
+    return out
+
+
 def _cuda(*ts):
     for t in ts:
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
@@ -192,8 +201,7 @@ def paged_attention_decode(q, k_pages, v_pages, block_tables, context_lens, scal
         raise ValueError("shape mismatch")
     if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
         raise TypeError("block_tables and context_lens must be int32")
-    if out is None:
-        out = torch.empty_like(q)
+    out = _out_like(q, out)
     MP = block_tables.shape[1]
     kv_dt = k_pages.dtype
     if workspace is None:
@@ -219,8 +227,7 @@ def paged_attention_decode_noalloc(q, k_pages, v_pages, block_tables, context_le
     _cuda(q, k_pages, v_pages, block_tables, context_lens, k_scales, v_scales, out)
     B, Hq, D = q.shape
     P, ps, Hkv, _ = k_pages.shape
-    if out is None:
-        out = torch.empty_like(q)
+    out = _out_like(q, out)
     _check(load().pkv_paged_attention_decode_noalloc(
         _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_tables), _ptr(context_lens), float(scale), _ptr(out),
         B, Hq, Hkv, D, ps, block_tables.shape[1], P, _dtype_code(q), _dtype_code(k_pages), _ptr(k_scales),
@@ -240,8 +247,7 @@ def paged_attention_prefill(q, k_pages, v_pages, block_tables, q_start, context_
     B = context_lens.shape[0]
     if D2 != D or q_start.shape[0] != B + 1:
         raise ValueError("shape mismatch")
-    if out is None:
-        out = torch.empty_like(q)
+    out = _out_like(q, out)
     if max_q_len is None:
         max_q_len = int((q_start[1:] - q_start[:-1]).max().item()) if B else 0
     lib = load()
