@@ -61,12 +61,16 @@ TRAFFIC = {
     "llama2_7b_mha_decode": {"bytes": 2363970000, "kernel_sha": "b47d14b81414f9e0"},
     # prefill_tc_kernel: 54.66 MB read + 4.87 MB written per launch, full workload, cold L2
     "chunked_prefill_shared_prefix": {"bytes": 59527936, "kernel_sha": "bf153121dbf992a1"},
+    # kv_scatter_kernel: 1120.62 MB per launch at a source batch of 16 (35 476 rows; ~43 MB of the
+    # writes still in L2 at the end), scaled to the 143 153-row launch by rows
+    "kv_cache_write_full": {"bytes": 4521850000, "kernel_sha": "d05e87c4610560d2"},
 }
 KERNEL_SOURCES = {
     "decode": ["paged_kv_cache_380_b200/csrc/decode.cu", "paged_kv_cache_380_b200/csrc/pkv_ptx.cuh",
                "paged_kv_cache_380_b200/csrc/pkv_common.cuh"],
     "prefill": ["paged_kv_cache_380_b200/csrc/prefill.cu", "paged_kv_cache_380_b200/csrc/pkv_ptx.cuh",
                 "paged_kv_cache_380_b200/csrc/pkv_common.cuh"],
+    "scatter": ["paged_kv_cache_380_b200/csrc/scatter.cu", "paged_kv_cache_380_b200/csrc/pkv_common.cuh"],
 }
 
 
