@@ -21,7 +21,7 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr int kChunk = 16;
 #ifndef PKV_SPLIT_MAX_CHUNKS
-#define PKV_SPLIT_MAX_CHUNKS 64   // longest automatic partition: 64 chunks of 16 tokens
+#define PKV_SPLIT_MAX_CHUNKS 128  // longest automatic partition: 128 chunks of 16 tokens (2048)
 #endif
 
 DeviceStatus* status_ptr() {

@@ -49,11 +49,11 @@ def test_error_strings(lib):
 
 def test_split_planner_on_the_workloads(lib):
     # Llama-2-7B decode: contexts up to 4096 tokens (256 pages of 16)
-    assert ops.decode_plan(64, 32, 32, 128, 16, 256) == (4, 1024)
+    assert ops.decode_plan(64, 32, 32, 128, 16, 256) == (2, 2048)
     # Llama-2-70B GQA decode: up to 8192 tokens
-    assert ops.decode_plan(128, 64, 8, 128, 16, 512) == (8, 1024)
-    # long context: 131072 tokens in 512 pages of 256 -> 128 partitions of 4 pages
-    assert ops.decode_plan(4, 32, 8, 128, 256, 512, torch.int8) == (128, 1024)
+    assert ops.decode_plan(128, 64, 8, 128, 16, 512) == (4, 2048)
+    # long context: 131072 tokens in 512 pages of 256 -> 64 partitions of 8 pages
+    assert ops.decode_plan(4, 32, 8, 128, 256, 512, torch.int8) == (64, 2048)
     # few (sequence, head) units -> shorter partitions, never below 256 tokens
     s, t = ops.decode_plan(1, 8, 1, 128, 16, 64)
     assert t == 256 and s == 4
