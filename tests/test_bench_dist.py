@@ -75,3 +75,25 @@ def test_reference_arm_line_shape(capsys, monkeypatch):
     assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+
+
+def test_reference_arm_cache_append_line(capsys, monkeypatch):
+    """The cache-append workload's reference arm: the oracle's row copy of a full-cache
+    scatter (here of a small decode batch standing in for the Llama-2-7B one)."""
+    import json
+
+    import numpy as np
+
+    import bench
+    from paged_kv_cache_380_b200 import workloads as W
+    small = W.decode_case(name="small_c2", config_index=1, batch=3, num_q_heads=4, num_kv_heads=4, head_dim=128,
+                          page_size=16, dtype="bf16", context_lens=np.array([17, 64, 300]))
+    monkeypatch.setattr(W, "llama2_7b_mha_decode", lambda **kw: small)
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    bench.run_reference(type("A", (), {"workload": "kv_cache_write_full", "steps": 2, "warmup": 3,
+                                       "ref_seqs": 1, "ref_items": 8})())
+    line = json.loads(capsys.readouterr().out.strip())
+    assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
+    assert line["dtype"] == "u8" and line["config"]["workload"] == "kv_cache_write_full"
+    assert line["cpu_baseline"]["kind"] == "oracle" and "381 rows" in line["cpu_baseline"]["sample"]
