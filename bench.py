@@ -60,7 +60,7 @@ TRAFFIC = {
     # algorithmic bytes; scaled to the batch-64 launch by algorithmic bytes (2346.50 MB)
     "llama2_7b_mha_decode": {"bytes": 2367850000, "kernel_sha": "0a93fece9ecd1e1c"},
     # prefill_tc_kernel: 54.66 MB read + 4.87 MB written per launch, full workload, cold L2
-    "chunked_prefill_shared_prefix": {"bytes": 59527936, "kernel_sha": "bf153121dbf992a1"},
+    "chunked_prefill_shared_prefix": {"bytes": 59527936, "kernel_sha": "1e682f307657a38b"},
     # kv_scatter_kernel: 1120.62 MB per launch at a source batch of 16 (35 476 rows; ~43 MB of the
     # writes still in L2 at the end), scaled to the 143 153-row launch by rows
     "kv_cache_write_full": {"bytes": 4521850000, "kernel_sha": "d05e87c4610560d2"},

@@ -310,6 +310,16 @@ int pkv_copy_pages(void* k_pages, void* v_pages, const int32_t* src, const int32
  */
 int pkv_get_device_status(pkv_stream_t stream, int64_t* detail);
 
+/*
+ * Self-test of the device time-out path (no counterpart on the pages).  Launches
+ * one thread that waits, with the bounded mbarrier wait the prefill kernel uses
+ * (1 s of %globaltimer), on a barrier that nothing ever completes.  The wait runs
+ * out, PKV_ERR_DEVICE_TIMEOUT is recorded in the device status word and the
+ * kernel returns; the context stays usable.  Read the result with
+ * pkv_get_device_status.  Returns PKV_OK once launched.
+ */
+int pkv_selftest_wait_timeout(pkv_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

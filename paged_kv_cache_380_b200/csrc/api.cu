@@ -287,6 +287,12 @@ int pkv_paged_attention_prefill(const void* q, const void* k_pages, const void* 
                                           page_size, max_pages_per_seq, num_pages, dtype, 0, stream);
 }
 
+int pkv_selftest_wait_timeout(pkv_stream_t stream) {
+    DeviceStatus* st = status_ptr();
+    if (!st) return PKV_ERR_CUDA;
+    return from_cuda(launch_wait_timeout_selftest(st, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int pkv_paged_attention_prefill_ex(const void* q, const void* k_pages, const void* v_pages,
                                    const int32_t* block_tables, const int32_t* q_start,
                                    const int32_t* context_lens, int causal, float scale, void* out,

@@ -70,5 +70,7 @@ struct PrefillParams {
 };
 
 cudaError_t launch_prefill(const PrefillParams& p, pkv_dtype dtype, cudaStream_t stream);
+// One bounded mbarrier wait that nothing completes (records PKV_ERR_DEVICE_TIMEOUT).
+cudaError_t launch_wait_timeout_selftest(DeviceStatus* st, cudaStream_t stream);
 
 }  // namespace pkv

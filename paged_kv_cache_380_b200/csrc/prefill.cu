@@ -544,6 +544,29 @@ cudaError_t run(const PrefillParams& p, cudaStream_t stream) {
 
 }  // namespace
 
+namespace {
+// One thread waits, with the prefill kernel's own bounded wait, on an mbarrier
+// that nothing ever arrives on: after kWaitLimitNs it records
+// PKV_ERR_DEVICE_TIMEOUT and the kernel returns.  Exercises the time-out path
+// without any fault or hang.
+__global__ void wait_timeout_selftest_kernel(DeviceStatus* st) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(ptx::smem_u32(&bar), 1);
+        abort_flag = 0;
+        ptx::fence_mbarrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) wait_bar(ptx::smem_u32(&bar), 0, &abort_flag, st);
+}
+}  // namespace
+
+cudaError_t launch_wait_timeout_selftest(DeviceStatus* st, cudaStream_t stream) {
+    wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(st);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_prefill(const PrefillParams& p, pkv_dtype dtype, cudaStream_t stream) {
     if (p.max_q_len <= 0 || p.num_seqs <= 0 || p.total_q <= 0) return cudaSuccess;
     return dtype == PKV_BF16 ? run<__nv_bfloat16>(p, stream) : run<__half>(p, stream);

@@ -30,7 +30,7 @@ EXPORTS = ("pkv_error_string", "pkv_kv_cache_write", "pkv_kv_cache_write_quant",
            "pkv_paged_attention_prefill",
            "pkv_get_device_status", "pkv_bm_create", "pkv_bm_destroy", "pkv_bm_add_sequence", "pkv_bm_fork",
            "pkv_bm_append", "pkv_bm_free_sequence", "pkv_bm_block_tables", "pkv_bm_num_free_pages",
-           "pkv_bm_page_refcount", "pkv_bm_num_sequences", "pkv_copy_pages")
+           "pkv_bm_page_refcount", "pkv_bm_num_sequences", "pkv_copy_pages", "pkv_selftest_wait_timeout")
 
 
 class PagedKVError(RuntimeError):
@@ -77,6 +77,8 @@ def load(path: str = _LIB_PATH):
         lib.pkv_paged_attention_prefill.restype = I
         lib.pkv_get_device_status.argtypes = [P, ctypes.POINTER(I64)]
         lib.pkv_get_device_status.restype = I
+        lib.pkv_selftest_wait_timeout.argtypes = [P]
+        lib.pkv_selftest_wait_timeout.restype = I
         lib.pkv_bm_create.argtypes = [I64, I, I]
         lib.pkv_bm_create.restype = P
         lib.pkv_bm_destroy.argtypes = [P]
@@ -259,6 +261,12 @@ def paged_attention_prefill(q, k_pages, v_pages, block_tables, q_start, context_
     else:
         _check(lib.pkv_paged_attention_prefill(*args, _stream(stream)), "paged_attention_prefill")
     return out
+
+
+def selftest_wait_timeout(stream=None) -> None:
+    """Launch a bounded wait that nothing completes (about 1 s); the device status
+    word then holds PKV_ERR_DEVICE_TIMEOUT."""
+    _check(load().pkv_selftest_wait_timeout(_stream(stream)), "selftest_wait_timeout")
 
 
 def device_status(stream=None):
