@@ -58,7 +58,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 TRAFFIC = {
     # decode_mma_kernel: 586.82 MB per launch at batch 16 (the capture-size case), 1.0091 x its
     # algorithmic bytes; scaled to the batch-64 launch by algorithmic bytes (2346.50 MB)
-    "llama2_7b_mha_decode": {"bytes": 2367850000, "kernel_sha": "0a93fece9ecd1e1c"},
+    "llama2_7b_mha_decode": {"bytes": 2367850000, "kernel_sha": "22b9d62d2b0642b1"},
     # prefill_tc_kernel: 54.66 MB read + 4.87 MB written per launch, full workload, cold L2
     "chunked_prefill_shared_prefix": {"bytes": 59527936, "kernel_sha": "1e682f307657a38b"},
     # kv_scatter_kernel: 1120.62 MB per launch at a source batch of 16 (35 476 rows; ~43 MB of the
