@@ -37,7 +37,9 @@
  *   - local (sliding-window) attention, the window_size argument of the
  *     attention call in [KVFA] §5.1 ("局部注意力"): with window w > 0 a query at
  *     position pos only sees keys pos-w+1 .. pos (keys below 0 do not exist);
- *     w <= 0 means no window.  Decode's query sits at pos = ctx-1.
+ *     w <= 0 means no window.  Decode's query sits at pos = ctx-1.  The pages
+ *     show the window only with causal masking; without it the window bounds
+ *     the lower side alone (keys pos-w+1 .. ctx-1).
  *   - symmetric INT8 quantisation of a K/V row ([SYS] §3.2 "量化压缩的工程实践",
  *     bits = 8, one group = one (token, KV head) row):  a = max|x| (fp32),
  *     scale = fp16(a / 127) (round to nearest even), code =

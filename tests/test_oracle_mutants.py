@@ -33,6 +33,9 @@ MUTANTS = [
     ("scatter_swaps_kv", "(const char*)v + t * row_bytes", "(const char*)k + t * row_bytes"),
     ("window_off_by_one", "pos - window + 1 > 0) ? pos - window + 1 : 0", "pos - window > 0) ? pos - window : 0"),
     ("decode_window_ignored", "(window > 0 && ctx - window > 0) ? ctx - window : 0", "0"),
+    ("window_only_when_causal", "int k_lo = (window > 0 && pos", "int k_lo = (window > 0 && causal && pos"),
+    ("window_band_from_context_end", "pos - window + 1 > 0) ? pos - window + 1 : 0",
+     "k_hi - window > 0) ? k_hi - window : 0"),
 ]
 
 CHECKS = [
@@ -60,7 +63,8 @@ CHECKS = [
     pins.test_bf16_widening_matches_torch_for_all_patterns,
     pins.test_window_covering_the_context_equals_no_window,
     pins.test_window_one_returns_the_own_value,
-    lambda: pins.test_window_matches_sdpa_band_mask(3),
+    lambda: pins.test_window_matches_sdpa_band_mask(3, True),
+    lambda: pins.test_window_matches_sdpa_band_mask(3, False),
 ]
 
 

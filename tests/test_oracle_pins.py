@@ -435,11 +435,14 @@ def test_window_one_returns_the_own_value():
             assert np.array_equal(out[b, h], v_last[h // 2])
 
 
+@pytest.mark.parametrize("causal", [True, False])
 @pytest.mark.parametrize("window", [1, 3, 6])
-def test_window_matches_sdpa_band_mask(window):
+def test_window_matches_sdpa_band_mask(window, causal):
+    """A query at position pos sees the window's w keys pos-w+1 .. pos when causal; without
+    the causal mask the window bounds only the lower side, so it sees pos-w+1 .. ctx-1."""
     rng = np.random.default_rng(32)
     c, q, qs, ctx = _prefill_case(rng)
-    out = oracle.prefill(q, "f64", c["k"], c["v"], "f64", c["bt"], qs, ctx, True, 0.35, window=window)
+    out = oracle.prefill(q, "f64", c["k"], c["v"], "f64", c["bt"], qs, ctx, causal, 0.35, window=window)
     Hq, Hkv = 4, 2
     for b in range(len(ctx)):
         n, L = int(qs[b + 1] - qs[b]), int(ctx[b])
@@ -448,7 +451,9 @@ def test_window_matches_sdpa_band_mask(window):
         Q = torch.from_numpy(q[qs[b]:qs[b + 1]]).permute(1, 0, 2)
         pos = (L - n + torch.arange(n))[:, None]
         key = torch.arange(L)[None, :]
-        mask = (key <= pos) & (key > pos - window)
+        mask = key > pos - window
+        if causal:
+            mask = mask & (key <= pos)
         ref = torch.nn.functional.scaled_dot_product_attention(Q, K, V, attn_mask=mask, scale=0.35)
         got = torch.from_numpy(out[qs[b]:qs[b + 1]]).permute(1, 0, 2)
         assert (got - ref).abs().max().item() < 1e-12
