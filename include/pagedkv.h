@@ -213,6 +213,11 @@ int pkv_paged_attention_prefill_ex(const void* q, const void* k_pages, const voi
  *   - All calls share the one array: calls that overlap on the GPU (several
  *     streams or host threads) race on it and must be serialised by the caller.
  *     Its contents persist between calls; no part of it needs to start zeroed.
+ *   - The looked-up address is kept for the life of the process.  A
+ *     cudaDeviceReset (or anything else that destroys the device's primary
+ *     context) unloads the array with the module, so that address, like the
+ *     cached address of the device status word, is stale afterwards: do not
+ *     call into the library on a device after resetting it in this process.
  * The library allocates no device memory on this path either.
  */
 #define PKV_NOALLOC_SCRATCH_BYTES (48u * 1024u * 1024u)

@@ -97,3 +97,27 @@ def test_reference_arm_cache_append_line(capsys, monkeypatch):
     assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
     assert line["dtype"] == "u8" and line["config"]["workload"] == "kv_cache_write_full"
     assert line["cpu_baseline"]["kind"] == "oracle" and "381 rows" in line["cpu_baseline"]["sample"]
+
+
+def test_cpu_baseline_reports_all_cores_and_one_thread():
+    """cpu_baseline times the oracle twice: on all host threads and on one."""
+    import numpy as np
+
+    import bench
+    import oracle
+    from paged_kv_cache_380_b200 import workloads as W
+    threads = oracle.max_threads()
+    dec = W.tiny_decode_f32()
+    step = type("S", (), {"case": dec, "kind": "decode", "int8": False, "has_new": False,
+                          "decode_bytes": 1e6})()
+    got = bench.cpu_baseline(step, budget_s=0.2)
+    assert got["cores"] == threads and got["value"] > 0
+    assert got["single_thread"]["cores"] == 1 and got["single_thread"]["value"] > 0
+    assert oracle.max_threads() == threads                 # thread count restored
+    pre = W.prefill_case(name="cpu_baseline_prefill", config_index=900, num_seqs=2, num_q_heads=4,
+                         num_kv_heads=2, head_dim=128, page_size=16, dtype="bf16", shared_prefix=16,
+                         chunk_lens=np.array([20, 9]), private_prefix=0)
+    step = type("S", (), {"case": pre, "kind": "prefill", "work": 1e9})()
+    got = bench.cpu_baseline(step, budget_s=0.2)
+    assert got["unit"] == "TFLOP/s" and got["single_thread"]["cores"] == 1
+    assert oracle.max_threads() == threads

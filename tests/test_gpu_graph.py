@@ -1,10 +1,12 @@
-"""GPU: the decode step captured in a CUDA graph equals the eager launches
-bit for bit, also after the inputs are updated in place between replays."""
+"""GPU: the decode step captured in a CUDA graph matches the fp64 oracle
+(max abs error 2e-2, bf16) and equals the eager launches bit for bit, also
+after the inputs are updated in place between replays."""
 import numpy as np
 import pytest
 import torch
 
-from gpu_util import assert_status_ok, dev
+import oracle
+from gpu_util import assert_close, assert_status_ok, dev, f64, host_bits
 from paged_kv_cache_380_b200 import ops
 from paged_kv_cache_380_b200 import workloads as W
 from paged_kv_cache_380_b200.graph import DecodeStepGraph
@@ -27,11 +29,17 @@ def test_graph_replay_matches_eager_and_follows_updates():
         ops.kv_cache_write(kn, vn, sl, kp_e, vp_e)
         return ops.paged_attention_decode(q, kp_e, vp_e, bt, cl, c.scale)
 
+    k_host, v_host = c.k_pages.copy(), c.v_pages.copy()
     for step in range(3):
         got = g.replay().clone()
         want = eager()
         torch.cuda.synchronize()
         assert_status_ok()
+        # the oracle: the same append, then decode, on host copies of this step's inputs
+        oracle.kv_cache_write(host_bits(kn), host_bits(vn), c.slot_mapping, k_host, v_host)
+        ref = oracle.decode(host_bits(q), "bf16", k_host, v_host, "bf16", c.block_tables,
+                            cl.cpu().numpy(), c.scale)
+        assert_close(f64(got), ref, 2e-2, f"graph replay, step {step}")
         assert torch.equal(got.view(torch.int16), want.view(torch.int16)), f"step {step}"
         assert torch.equal(kp_g.view(torch.int16), kp_e.view(torch.int16))
         # next step: new queries, one sequence shorter, another's newest row rewritten
