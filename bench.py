@@ -60,6 +60,12 @@ TRAFFIC = {
     # decode_mma_kernel: 586.82 MB per launch at batch 16 (the capture-size case), 1.0091 x its
     # algorithmic bytes; scaled to the batch-64 launch by algorithmic bytes (2346.50 MB)
     "llama2_7b_mha_decode": {"bytes": 2367850000, "kernel_sha": "22b9d62d2b0642b1"},
+    # decode_mma_kernel (GQA, 8 query heads per KV head): 317.67 MB per launch at batch 32 (the
+    # capture-size case), 1.012 x its algorithmic bytes; scaled to the batch-128 launch (1396.15 MB)
+    "llama2_70b_gqa_decode": {"bytes": 1412900000, "kernel_sha": "22b9d62d2b0642b1"},
+    # decode_mma_kernel (int8 codes + fp16 scales): 281.64 MB per launch at batch 1 (the capture-size
+    # case), 1.033 x its algorithmic bytes (split partials included); scaled to batch 4 (1090.59 MB)
+    "long_ctx_split_kv_int8": {"bytes": 1126600000, "kernel_sha": "22b9d62d2b0642b1"},
     # prefill_tc_kernel: 54.66 MB read + 4.87 MB written per launch, full workload, cold L2
     "chunked_prefill_shared_prefix": {"bytes": 59527936, "kernel_sha": "1e682f307657a38b"},
     # kv_scatter_kernel: 1120.62 MB per launch at a source batch of 16 (35 476 rows; ~43 MB of the
