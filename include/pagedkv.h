@@ -245,7 +245,9 @@ int pkv_paged_attention_decode_noalloc(const void* q, const void* k_pages, const
  *   q_start    int32 [num_seqs + 1], q_start[0] = 0, nondecreasing,
  *              q_start[num_seqs] = total_q
  *   max_q_len  >= every n_b (sizes the launch grid)
- *   head_dim   128; page_size a multiple of 16
+ *   scale      the softmax scale, finite and > 0 (1/sqrt(head_dim) on the
+ *              pages); anything else is PKV_ERR_INVALID_ARG
+ *   head_dim   64 or 128; page_size a multiple of 16
  *   q, out, k_pages, v_pages 16-byte aligned (else PKV_ERR_INVALID_ARG)
  * n_b > context_lens[b] is recorded as a device range error.
  */

@@ -302,14 +302,15 @@ int pkv_paged_attention_prefill_ex(const void* q, const void* k_pages, const voi
                                    int head_dim, int page_size, int max_pages_per_seq, int64_t num_pages,
                                    pkv_dtype dtype, int window, pkv_stream_t stream) {
     if (num_seqs < 0 || total_q < 0 || max_q_len < 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
-        head_dim <= 0 || page_size <= 0 || max_pages_per_seq <= 0 || num_pages <= 0 || !std::isfinite(scale))
+        head_dim <= 0 || page_size <= 0 || max_pages_per_seq <= 0 || num_pages <= 0 || !std::isfinite(scale) ||
+        !(scale > 0.f))
         return PKV_ERR_INVALID_ARG;
     if (num_q_heads % num_kv_heads) return PKV_ERR_INVALID_ARG;
     if (num_seqs == 0 || total_q == 0 || max_q_len == 0) return PKV_OK;
     if (!q || !k_pages || !v_pages || !block_tables || !q_start || !context_lens || !out)
         return PKV_ERR_INVALID_ARG;
     if (dtype != PKV_BF16 && dtype != PKV_F16) return PKV_ERR_UNSUPPORTED;
-    if (head_dim != 128 || page_size % kChunk) return PKV_ERR_UNSUPPORTED;
+    if ((head_dim != 64 && head_dim != 128) || page_size % kChunk) return PKV_ERR_UNSUPPORTED;
     // q and the pools are TMA tensor-map bases; out is written with 16-byte stores
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16))
         return PKV_ERR_INVALID_ARG;

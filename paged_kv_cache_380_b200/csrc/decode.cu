@@ -80,6 +80,10 @@ struct DecodeCfg {
     static constexpr int kMerge = WARPS * 8 * NT * (HD + 2) * 4;
     static constexpr int kSmem = kPipe > kMerge ? kPipe : kMerge;
     static constexpr int kDT = HD / 16;   // 16-wide d tiles (MMA k-steps for QK, M tiles for PV)
+    // Lazy rescale: probabilities are taken against a reference max that may lag the
+    // running max by up to 2^kRescale (P <= 256 in the bf16 / fp16 MMA operand).  The
+    // INT8 path multiplies P by the value scale in fp16, so it keeps P <= 1 there.
+    static constexpr float kRescale = kInt8 ? 0.f : 8.f;
     static_assert(kUnits >= 8, "rows must span at least 128 bytes for the swizzle");
     static_assert(!kInt8 || HD == 128, "INT8 pages need head_dim 128");
 };
@@ -93,7 +97,9 @@ decode_mma_kernel(const DecodeParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
-    const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+    // partitions vary slowest: every sequence's first (longest) partitions are
+    // dispatched before the partial remainders, which then fill the tail
+    const int kvh = blockIdx.x, b = blockIdx.y, split = blockIdx.z;
     const int Hq = p.num_q_heads, Hkv = p.num_kv_heads, G = Hq / Hkv, ps = p.page_size;
 
     const int ctx = __ldg(p.context_lens + b);
@@ -298,17 +304,22 @@ decode_mma_kernel(const DecodeParams p) {
                 mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
                 mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
                 mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
-                const float m_new = fmaxf(m[nt][h], mx);   // finite: every chunk holds an attended token
-                const float corr = ptx::ex2(m[nt][h] - m_new);
-                m[nt][h] = m_new;
-                pr[h] = ptx::ex2(x[h] - m_new);
-                pr[2 + h] = ptx::ex2(x[2 + h] - m_new);
-                l[nt][h] = l[nt][h] * corr + (pr[h] + pr[2 + h]);
+                // m is a reference max: the accumulator is rescaled only when the chunk's
+                // max exceeds it by more than kRescale (finite: every chunk holds an
+                // attended token; the first chunk always rescales from -inf)
+                if (mx > m[nt][h] + Cfg::kRescale) {
+                    const float corr = ptx::ex2(m[nt][h] - mx);
+                    m[nt][h] = mx;
+                    l[nt][h] *= corr;
 #pragma unroll
-                for (int dt = 0; dt < Cfg::kDT; ++dt) {
-                    o[nt][dt][h] *= corr;
-                    o[nt][dt][2 + h] *= corr;
+                    for (int dt = 0; dt < Cfg::kDT; ++dt) {
+                        o[nt][dt][h] *= corr;
+                        o[nt][dt][2 + h] *= corr;
+                    }
                 }
+                pr[h] = ptx::ex2(x[h] - m[nt][h]);
+                pr[2 + h] = ptx::ex2(x[2 + h] - m[nt][h]);
+                l[nt][h] += pr[h] + pr[2 + h];
             }
             // P^T fragments (B operand of O^T += V^T . P^T) via 8x8 transposes
             pb[nt][0] = ptx::movmatrix_trans(pack2<MT>(pr[0] * vs_a, pr[1] * vs_a));
@@ -543,7 +554,7 @@ cudaError_t run_mma(const DecodeParams& p, cudaStream_t stream) {
     auto kern = decode_mma_kernel<QT, KVT, HD, NT, kWarps, kStages>;
     cudaError_t e0 = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), Cfg::kSmem);
     if (e0 != cudaSuccess) return e0;
-    dim3 grid(p.max_splits, p.num_kv_heads, p.num_seqs);
+    dim3 grid(p.num_kv_heads, p.num_seqs, p.max_splits);
     kern<<<grid, kWarps * 32, Cfg::kSmem, stream>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || p.max_splits == 1) return e;

@@ -11,27 +11,35 @@
 // Flash Attention，让 Token 生成快 3 倍" ("Flash Attention 的分块计算原理"),
 // K/V read page by page through the block table.
 //
-// B200 design, one CTA per (128-row query tile, query head, sequence), 12 warps:
-//  * warps 0-2 = TMA producers: the Q tile once (two 64-column SW128 boxes), then
-//    per 128-key tile one 16-row box per page group and 64-column half for K and
-//    for V (lane pairs of the three warps split the 16 boxes of a tile), into
-//    rings of 3 K stages and 2 V stages (mbarrier expect_tx).
-//  * warp 3 = MMA issuer (one thread): S_j = Q K_j^T (M=128, N=128, K=128, bf16
-//    -> fp32 in TMEM, three S/P buffers) and O += P_j V_j with P read from TMEM
-//    (the TS form) and V as an MN-major operand.  S runs two tiles ahead of PV
-//    (S_0 S_1 | PV_0 S_2 | PV_1 S_3 ...), so the softmax of tile i+1 never waits
-//    for P_i.  One tcgen05.commit per MMA group (each commit costs tensor-pipe
-//    time): "S_j done" also frees K stage j, "PV_i done" also frees P buffer i
-//    and the V stage PV_i read.
-//  * warps 4-11 = softmax: one TMEM lane (query row) per thread, two warps per
-//    row quarter taking 64 columns each (row max and row sum exchanged in
-//    shared memory); tcgen05.ld of the S half-row, masking, max, 2^(s*scale -
-//    m) with the scale folded into one FFMA, row sum, P packed to bf16 pairs
-//    and tcgen05.st back over the S columns; one P-ready arrival per warp.  The
-//    accumulator is rescaled only when a row's running max grows by more than
-//    2^8 (P <= 256 otherwise), which keeps O's TMEM round trip off most tiles;
-//    the final division by the row sum makes any consistent reference max exact.
-//  * Heaviest (longest causal) query tiles are launched first.
+// B200 design.  One CTA of 12 warps per (128-row query tile, pair of query
+// heads, sequence).  The two query heads of a pair read the same KV head
+// (grouped-query attention, "LLM推理系统优化：KV缓存管理与动态批处理技术"
+// §2.1), so they share the causal mask, the key range and every K/V tile: each
+// tile is loaded once and feeds two S tiles and two PV tiles.  The two query
+// tiles ("A" and "B") form a ping-pong: while the softmax of one runs on the
+// CUDA cores, the tensor pipe works on the other.
+//  * TMEM (512 columns): S_A | S_B | O_A | O_B, 128 columns each.  P (bf16)
+//    overwrites the first half of its own S tile.
+//  * warp 0 = K producer, warp 1 = V producer: per 128-key tile, one 16-row TMA
+//    box per page group and 64-column half (one box per lane), into rings of 3
+//    K stages and 2 V stages (mbarrier expect_tx).  Warp 0 also loads both Q
+//    tiles once.
+//  * warp 2 = MMA issuer (one thread), per key tile j:
+//        PV_A(j)  S_A(j+1)  PV_B(j)  S_B(j+1)
+//    S = Q K^T (M=128, N=128, both operands K-major in shared memory), PV = P V
+//    with P read from TMEM (the TS form) and V as an MN-major operand.  Issuing
+//    S_X(j+1) right behind PV_X(j) is what lets P alias S: tcgen05 MMAs of one
+//    thread execute in issue order.  Each commit signals one barrier: "S_B(j)
+//    done" also frees K stage j, "PV_B(j) done" also frees V stage j.
+//  * warps 4-7 = softmax of tile A, warps 8-11 = softmax of tile B: one TMEM
+//    lane (query row) per thread, all 128 columns of its row.  tcgen05.ld of
+//    the S row, masking, row max, 2^(s*scale - m) with the scale folded into one
+//    FFMA, row sum, P packed to bf16 pairs and tcgen05.st over the S columns;
+//    one P-ready arrival per warp.  The accumulator is rescaled only when a
+//    row's running max grows by more than 2^8 (P <= 256 otherwise); the final
+//    division by the row sum makes any consistent reference max exact.
+//  * Heads of a group that cannot be paired (an odd group size) run one tile
+//    per CTA through the same code (NT = 1).
 //  * Every mbarrier wait polls (test_wait) and is bounded in time; on time-out
 //    the CTA records PKV_ERR_DEVICE_TIMEOUT, raises an abort flag so every role
 //    leaves its loop, waits (bounded) for its own async work and frees TMEM.
@@ -39,7 +47,6 @@
 
 #include <cmath>
 #include <cstring>
-#include <mutex>
 #include <type_traits>
 
 #include "pkv_kernels.h"
@@ -48,31 +55,49 @@
 namespace pkv {
 namespace {
 
-constexpr int BM = 128, BN = 128, HD = 128;
-constexpr int KST = 3, VST = 2, NSB = 3;        // K stages, V stages, S/P TMEM buffers
-constexpr int kProducerWarps = 3;               // TMA issue is split over three warps
-constexpr int kMmaWarp = kProducerWarps;
-constexpr int kSoftmaxWarp0 = kMmaWarp + 1;
-constexpr int kSoftmaxWarps = 8;                // two warps per TMEM lane quarter, 64 columns each
-constexpr int kThreads = (kSoftmaxWarp0 + kSoftmaxWarps) * 32;   // 12 warps = 3 warpgroups
-constexpr int kAtom = BN * 128;                 // one 64-column SW128 half of a 128-row tile
-constexpr int kTile = 2 * kAtom;                // 32 KB
-constexpr int kSmemQ = 0;
-constexpr int kSmemK = kSmemQ + kTile;
-constexpr int kSmemV = kSmemK + KST * kTile;
-constexpr int kSmemRed = kSmemV + VST * kTile;   // row-max / row-sum exchange between warp pairs
-constexpr int kRedBytes = (2 * 2 * BM + 2 * BM) * 4;
-constexpr int kSmemBar = kSmemRed + kRedBytes;
-constexpr int kNumBars = 1 + KST + VST + 3 * NSB + 1;
-constexpr int kSmemBytes = kSmemBar + kNumBars * 8 + 16 + 1024;   // + TMEM addr, abort flag, alignment
+constexpr int BM = 128, BN = 128;               // query rows / keys per tile
+constexpr int KST = 3, VST = 2;                 // K stages, V stages
+constexpr int kRing = 6;                        // KST and VST ring positions repeat every 6 key tiles
+constexpr int kKWarp = 0, kVWarp = 1, kMmaWarp = 2, kSoftWarp0 = 4;
+constexpr int kThreads = 12 * 32;               // 3 warpgroups
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kOCol = NSB * 128;           // O accumulator columns 384..511
+constexpr uint32_t kOCol = 256;                 // O of tile X at 256 + 128 X; S/P of tile X at 128 X
+constexpr int kAtom = BM * 128;                 // one 64-column SW128 atom of a 128-row tile (16 KB)
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // bound of every mbarrier wait (1 s)
 constexpr float kRescaleThreshold = 8.0f;       // log2 units: rescale when the max grows by > 2^8
 
-__device__ __forceinline__ void named_bar_sync(int id, int threads) {
-    asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");
-}
+// Shared-memory layout of the CTA for head_dim HD and NT query tiles.
+template <int HD, int NT>
+struct Layout {
+    static constexpr int NH = HD / 64;          // 64-column atoms per row
+    static constexpr int kTile = NH * kAtom;    // one 128-row tile of HD columns
+    static constexpr int kQ = 0;
+    static constexpr int kK = kQ + NT * kTile;
+    static constexpr int kV = kK + KST * kTile;
+    static constexpr int kBar = kV + VST * kTile;
+    static constexpr int kNumBars = 1 + KST + VST + 2 * KST + 2 + VST + 2 + 1;
+    static constexpr int kEnd = kBar + kNumBars * 8 + 16;   // + TMEM address, abort flag
+    // The CTA holds all of TMEM, so only one may run per SM: ask for more than
+    // half of the SM's shared memory even when the tiles need less.
+    static constexpr int kSmem = kEnd + 1024 > 120 * 1024 ? kEnd + 1024 : 120 * 1024;
+};
+
+// mbarriers, all in one array after the tiles.
+struct Bars {
+    uint32_t base;
+    __device__ __forceinline__ uint32_t at(int i) const { return base + 8 * i; }
+    __device__ __forceinline__ uint32_t q_full() const { return at(0); }
+    __device__ __forceinline__ uint32_t k_full(int s) const { return at(1 + s); }
+    __device__ __forceinline__ uint32_t v_full(int s) const { return at(1 + KST + s); }
+    // S_X(j) done (and, for the last tile, K stage s free), one barrier per K stage
+    __device__ __forceinline__ uint32_t s_full(int x, int s) const { return at(1 + KST + VST + x * KST + s); }
+    __device__ __forceinline__ uint32_t p_full(int x) const { return at(1 + 3 * KST + VST + x); }
+    // PV of the last tile done: V stage s free
+    __device__ __forceinline__ uint32_t pv_done(int s) const { return at(3 + 3 * KST + VST + s); }
+    __device__ __forceinline__ uint32_t o_full(int x) const { return at(3 + 3 * KST + 2 * VST + x); }
+    __device__ __forceinline__ uint32_t mma_done() const { return at(5 + 3 * KST + 2 * VST); }
+};
+static_assert(5 + 3 * KST + 2 * VST + 1 == 1 + KST + VST + 2 * KST + 2 + VST + 2 + 1, "barrier count");
 
 // sm_100 shared-memory matrix descriptor: start, leading and stride byte
 // offsets (>> 4), version 1, SWIZZLE_128B layout.
@@ -91,33 +116,55 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int b_mn_major) {
            (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// mbarrier addresses, all in one array after the tiles.  Every tcgen05.commit costs
-// tensor-pipe time, so each MMA group signals exactly one barrier: s_done(b) =
-// "S in buffer b is ready and K stage b is free" (K stages and S buffers share
-// the ring index), pv_done(b) = "O is updated, P buffer b and the V stage that
-// PV read are free".
-struct Bars {
-    uint32_t base;
-    __device__ __forceinline__ uint32_t q_full() const { return base; }
-    __device__ __forceinline__ uint32_t k_full(int i) const { return base + 8 * (1 + i); }
-    __device__ __forceinline__ uint32_t v_full(int i) const { return base + 8 * (1 + KST + i); }
-    __device__ __forceinline__ uint32_t s_done(int i) const { return base + 8 * (1 + KST + VST + i); }
-    __device__ __forceinline__ uint32_t p_full(int i) const { return base + 8 * (1 + KST + VST + NSB + i); }
-    __device__ __forceinline__ uint32_t pv_done(int i) const { return base + 8 * (1 + KST + VST + 2 * NSB + i); }
-    __device__ __forceinline__ uint32_t mma_done() const { return base + 8 * (1 + KST + VST + 3 * NSB); }
-};
+// Each thread of the warp writes 32 consecutive 32-bit columns of its own TMEM lane.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+        "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+// Each thread of the warp reads 16 consecutive 32-bit columns of its own TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+// Per-warpgroup register budget changes (all threads of a warpgroup execute them).
+template <int N>
+__device__ __forceinline__ void ptx_setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void ptx_setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+
+#ifndef PKV_PREFILL_MMA_SLEEP
+#define PKV_PREFILL_MMA_SLEEP 1
+#endif
 
 // Bounded wait that also gives up as soon as another role raised the abort flag.
-// It polls with the non-blocking test_wait: the pipeline is latency-bound, and a
-// thread suspended inside try_wait resumes measurably later than a polling one
-// (13% of the prefill time on a 128-row causal workload).  The bound is 1 s of
-// %globaltimer, after which the CTA records PKV_ERR_DEVICE_TIMEOUT.
+// kSleep: the thread waits inside try_wait, suspended until the phase completes
+// (or a hardware time slice ends), so a waiting warp takes no issue slots from
+// the working warps of its sub-partition.  Otherwise it polls with the
+// non-blocking test_wait.  The bound is 1 s of %globaltimer, after which the CTA
+// records PKV_ERR_DEVICE_TIMEOUT.
+template <bool kSleep = true>
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                          DeviceStatus* st) {
-    if (ptx::mbar_test_wait(bar, parity)) return true;
+    auto probe = [&] { return kSleep ? ptx::mbar_try_wait(bar, parity) : ptx::mbar_test_wait(bar, parity); };
+    if (probe()) return true;
     const uint64_t t0 = ptx::globaltimer_ns();
     for (;;) {
-        if (ptx::mbar_test_wait(bar, parity)) return true;
+        if (probe()) return true;
         if (*abort_flag) return false;
         if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) break;
     }
@@ -126,45 +173,108 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     return false;
 }
 
-// One S tile: S[buffer SB] = Q K[stage SB]^T (K stages and S buffers share the index).
-template <typename T, int SB>
-__device__ __forceinline__ void mma_s(uint32_t sbase, const Bars& bars) {
-    static_assert(KST == NSB, "K stage and S buffer share one ring index");
-    constexpr uint32_t id_s = idesc_f16<T>(BM, BN, 0);
-    const uint32_t kbase = sbase + kSmemK + SB * kTile;
-#pragma unroll
-    for (int kk = 0; kk < HD / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
-        ptx::tc_mma_ss(SB * 128, sdesc(sbase + kSmemQ + off, 16, 1024), sdesc(kbase + off, 16, 1024), id_s,
-                       kk > 0 ? 1u : 0u);
-    }
-    ptx::tc_commit(bars.s_done(SB));
-}
-// One PV tile: O (+)= P[buffer PB] V[stage VS]; ACC = false only for the first tile.
-template <typename T, int PB, int VS, bool ACC>
-__device__ __forceinline__ void mma_pv(uint32_t sbase, const Bars& bars) {
-    constexpr uint32_t id_o = idesc_f16<T>(BM, HD, 1);
-    const uint32_t vbase = sbase + kSmemV + VS * kTile;
-#pragma unroll
-    for (int kk = 0; kk < BN / 16; ++kk)
-        ptx::tc_mma_ts(kOCol, PB * 128 + kk * 8, sdesc(vbase + kk * 2048, kAtom, 1024), id_o,
-                       (ACC || kk > 0) ? 1u : 0u);
-    ptx::tc_commit(bars.pv_done(PB));
-}
+// The MMA issuer's view of the CTA: operand addresses are compile-time offsets
+// from the shared-memory base, and the ring slots are template arguments, so
+// every MMA operand is a constant.
+template <typename T, int HD, int NT>
+struct Issuer {
+    using L = Layout<HD, NT>;
+    uint32_t sbase;
+    Bars bars;
+    volatile int* abort_flag;
+    DeviceStatus* status;
 
-template <typename T>
+    __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity) const {
+        return wait_bar<PKV_PREFILL_MMA_SLEEP != 0>(bar, parity, abort_flag, status);
+    }
+    // The shared-memory base, opaque to the compiler: descriptors are rebuilt at
+    // each use (a few integer instructions) instead of being hoisted out of the
+    // key loop into dozens of live registers.
+    __device__ __forceinline__ uint32_t base() const {
+        uint32_t b;
+        asm volatile("mov.b32 %0, %1;\n" : "=r"(b) : "r"(sbase));
+        return b;
+    }
+    // S_X = Q_X K[stage KS]^T, then one commit: "S_X done" (+ K stage free for the last tile).
+    template <int X, int KS>
+    __device__ __forceinline__ void s() const {
+        constexpr uint32_t id = idesc_f16<T>(BM, BN, 0);
+        const uint32_t sb = base();
+        const uint32_t qa = sb + L::kQ + X * L::kTile, ka = sb + L::kK + KS * L::kTile;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
+            ptx::tc_mma_ss(X * 128, sdesc(qa + off, 16, 1024), sdesc(ka + off, 16, 1024), id, kk > 0 ? 1u : 0u);
+        }
+        ptx::tc_commit(bars.s_full(X, KS));
+    }
+    // O_X (+)= P_X V[stage VS]; the first key tile overwrites O.
+    template <int X, int VS>
+    __device__ __forceinline__ void pv(bool acc) const {
+        constexpr uint32_t id = idesc_f16<T>(BM, HD, 1);
+        const uint32_t va = base() + L::kV + VS * L::kTile;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+            ptx::tc_mma_ts(kOCol + X * 128, X * 128 + kk * 8, sdesc(va + kk * 2048, kAtom, 1024), id,
+                           (acc || kk > 0) ? 1u : 0u);
+    }
+    // Key tile j (R = j % kRing): PV_A(j) S_A(j+1) [PV_B(j) S_B(j+1)].
+    template <int R>
+    __device__ __forceinline__ bool step(int j, int n) const {
+        constexpr int VS = R % VST, KS1 = (R + 1) % KST;
+        const bool more = j + 1 < n;
+        if (!wait(bars.p_full(0), j & 1) || !wait(bars.v_full(VS), (j / VST) & 1)) return false;
+        ptx::tc_fence_after();
+        pv<0, VS>(j > 0);
+        if constexpr (NT == 1) ptx::tc_commit(bars.pv_done(VS));
+        if (!more) ptx::tc_commit(bars.o_full(0));
+        if (more) {
+            if (!wait(bars.k_full(KS1), ((j + 1) / KST) & 1)) return false;
+            ptx::tc_fence_after();
+            s<0, KS1>();
+        }
+        if constexpr (NT == 2) {
+            if (!wait(bars.p_full(1), j & 1)) return false;
+            ptx::tc_fence_after();
+            pv<1, VS>(j > 0);
+            ptx::tc_commit(bars.pv_done(VS));
+            if (!more) ptx::tc_commit(bars.o_full(1));
+            if (more) s<1, KS1>();
+        }
+        return true;
+    }
+    __device__ void run(int n) const {
+        if (!wait(bars.q_full(), 0) || !wait(bars.k_full(0), 0)) return;
+        ptx::tc_fence_after();
+        s<0, 0>();
+        if constexpr (NT == 2) s<1, 0>();
+        bool ok = true;
+        for (int j = 0; j < n && ok; ++j) {
+            switch (j % kRing) {
+            case 0: ok = step<0>(j, n); break;
+            case 1: ok = step<1>(j, n); break;
+            case 2: ok = step<2>(j, n); break;
+            case 3: ok = step<3>(j, n); break;
+            case 4: ok = step<4>(j, n); break;
+            default: ok = step<5>(j, n); break;
+            }
+        }
+    }
+};
+
+template <typename T, int HD, int NT>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
+    using L = Layout<HD, NT>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = ptx::smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    const int num_qt = gridDim.z;
-    const int qt = num_qt - 1 - static_cast<int>(blockIdx.z);   // heaviest tiles first
-    const int h = blockIdx.x, b = blockIdx.y;
-    const int Hq = p.num_q_heads, Hkv = p.num_kv_heads, kvh = h / (Hq / Hkv), ps = p.page_size;
+    const int qt = static_cast<int>(gridDim.z) - 1 - static_cast<int>(blockIdx.z);   // heaviest tiles first
+    const int h0 = blockIdx.x * NT, b = blockIdx.y;
+    const int Hq = p.num_q_heads, kvh = h0 / (Hq / p.num_kv_heads), ps = p.page_size;
     const int q0 = __ldg(p.q_start + b), n = __ldg(p.q_start + b + 1) - q0;
     const int ctx = __ldg(p.context_lens + b);
     const int r0 = qt * BM;
@@ -176,40 +286,33 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
     const int last_row = min(r0 + BM, n) - 1;
     const int max_key = p.causal ? ctx - n + last_row : ctx - 1;
     const int min_lim = p.causal ? ctx - n + r0 : ctx - 1;      // every row of the tile sees keys <= this
-    // Local attention (window w > 0): a row at position pos sees keys pos-w+1 .. pos,
-    // so the tile's key range starts at the first row's lower bound, and keys below
-    // the last row's lower bound need the lower-edge mask.
+    // Local attention (window w > 0): a row at position pos sees keys pos-w+1 .. pos
+    // (pos-w+1 .. ctx-1 without the causal mask), so the tile's key range starts at
+    // the first row's lower bound, and keys below the last row's lower bound need
+    // the lower-edge mask.
     const int w = p.window;
     const int key_lo = w > 0 ? max(0, ctx - n + r0 - w + 1) : 0;
     const int lo_mask = w > 0 ? max(0, ctx - n + last_row - w + 1) : 0;
     const int t_first = key_lo / BN;
     const int n_tiles = max_key / BN + 1 - t_first;
-    auto tile_of = [&](int j) { return t_first + j; };
 
-    const Bars bars{sbase + kSmemBar};
-    // Page indices, 4 tiles (32 groups of 16 keys) per batch: lane i of batch k holds the
-    // physical page of group i%8 of tile 4k + i/8 (loaded by the producer warp only).
-    const int32_t* bt = p.block_tables + static_cast<size_t>(b) * p.max_pages_per_seq;
-    auto load_pages = [&](int k) -> int {
-        const int key0 = tile_of(4 * k + (lane >> 3)) * BN + 16 * (lane & 7);
-        return key0 < ctx ? __ldg(bt + key0 / ps) : -1;
-    };
-    int pg_cur = 0, pg_next = 0;
-    if (warp < kProducerWarps) {
-        pg_cur = load_pages(0);
-        pg_next = load_pages(1);
-    }
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kSmemBar + kNumBars * 8);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSmemBar + kNumBars * 8 + 8);
+    const Bars bars{sbase + L::kBar};
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBar + L::kNumBars * 8);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kBar + L::kNumBars * 8 + 8);
 
     if (threadIdx.x == 0) {
         ptx::mbar_init(bars.q_full(), 1);
-        for (int i = 0; i < KST; ++i) ptx::mbar_init(bars.k_full(i), kProducerWarps);
-        for (int i = 0; i < VST; ++i) ptx::mbar_init(bars.v_full(i), kProducerWarps);
-        for (int i = 0; i < NSB; ++i) {
-            ptx::mbar_init(bars.s_done(i), 1);
-            ptx::mbar_init(bars.p_full(i), kSoftmaxWarps);
+        for (int i = 0; i < KST; ++i) {
+            ptx::mbar_init(bars.k_full(i), 1);
+            for (int x = 0; x < 2; ++x) ptx::mbar_init(bars.s_full(x, i), 1);
+        }
+        for (int i = 0; i < VST; ++i) {
+            ptx::mbar_init(bars.v_full(i), 1);
             ptx::mbar_init(bars.pv_done(i), 1);
+        }
+        for (int x = 0; x < 2; ++x) {
+            ptx::mbar_init(bars.p_full(x), 4);                  // one arrival per softmax warp
+            ptx::mbar_init(bars.o_full(x), 1);
         }
         ptx::mbar_init(bars.mma_done(), 1);
         *abort_flag = 0;
@@ -224,270 +327,215 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
     ptx::tc_fence_after();
     // All 512 columns are allocated, so the allocation starts at lane 0, column 0
     // and the MMAs use constant TMEM addresses; anything else is reported.
-    const uint32_t tmem = 0;
     if (threadIdx.x == 0 && *tmem_slot != 0u) {
         *abort_flag = 1;
         record_error(p.status, PKV_ERR_CUDA, static_cast<long long>(*tmem_slot));
     }
 
-    if (warp < kProducerWarps) {
+    // Register split (setmaxnreg acts per warpgroup): the producer / MMA warpgroup
+    // gives registers back so that each softmax thread can hold a whole S row.
+    // Launch: 384 threads x 168; after: 128 x 56 + 256 x 216 = 62464 <= 64512.
+    __syncwarp();
+    if (warp < 4) {
+    ptx_setmaxnreg_dec<56>();
+    if (warp == kKWarp || warp == kVWarp) {
         // ------------------------------ TMA producers ------------------------------
-        // A tile is 8 page groups x 2 column halves = 16 boxes per tensor; producer
-        // warp w issues the boxes of groups w, w+3, w+6 (one box per lane), because a
-        // single issuing warp cannot keep enough 2 KB boxes in flight.  K runs up to KST
-        // tiles ahead; V is issued one tile behind K so that waiting for a free V
-        // stage never delays the next K tile.  Page indices come from register
-        // batches loaded four tiles ahead (pg_cur / pg_next).
-        if (warp == 0 && lane == 0) {
-            ptx::prefetch_tmap(&tm_q);
-            ptx::prefetch_tmap(&tm_k);
-            ptx::prefetch_tmap(&tm_v);
-            ptx::mbar_arrive_expect_tx(bars.q_full(), kTile);
-            ptx::tma_load_3d(sbase + kSmemQ, &tm_q, bars.q_full(), 0, h, q0 + r0);
-            ptx::tma_load_3d(sbase + kSmemQ + kAtom, &tm_q, bars.q_full(), 64, h, q0 + r0);
+        // A key tile is 8 page groups of 16 rows x NH column atoms: one box per lane.
+        // K runs up to KST tiles ahead of the S MMAs, V up to VST tiles ahead of PV.
+        const bool is_k = warp == kKWarp;
+        const int nst = is_k ? KST : VST;
+        const CUtensorMap* map = is_k ? &tm_k : &tm_v;
+        const uint32_t ring = sbase + (is_k ? L::kK : L::kV);
+        if (lane == 0) {
+            ptx::prefetch_tmap(map);
+            if (is_k) {
+                ptx::prefetch_tmap(&tm_q);
+                ptx::mbar_arrive_expect_tx(bars.q_full(), NT * L::kTile);
+                for (int x = 0; x < NT; ++x)
+                    for (int a = 0; a < L::NH; ++a)
+                        ptx::tma_load_3d(sbase + L::kQ + x * L::kTile + a * kAtom, &tm_q, bars.q_full(), 64 * a,
+                                         h0 + x, q0 + r0);
+            }
         }
-        const int my_group = warp + kProducerWarps * (lane >> 1);   // lane pair -> one page group
-        const int my_half = lane & 1;
-        const bool my_lane = my_group < 8;
-        // TMA row (slot) of my page group in tile t, or -1 (past the context / bad page)
-        auto row_of = [&](int t, int pg_word) -> int {
-            const int page = __shfl_sync(0xffffffffu, pg_word, (t & 3) * 8 + (my_group & 7));
-            const int key0 = tile_of(t) * BN + 16 * my_group;
-            if (!my_lane || key0 >= ctx) return -1;
-            if (page < 0 || page >= p.num_pages) {
-                if (my_half == 0) record_error(p.status, PKV_ERR_DEVICE_RANGE, page);
-                return -1;
-            }
-            return page * ps + key0 % ps;
+        const int group = lane / L::NH, half = lane % L::NH;
+        const bool my_lane = group < 8;
+        const int32_t* bt = p.block_tables + static_cast<size_t>(b) * p.max_pages_per_seq;
+        // physical page of my group in tile t (read one tile ahead of its use), or -1
+        auto page_of = [&](int t) -> int {
+            const int key0 = (t_first + t) * BN + 16 * group;
+            return (my_lane && t < n_tiles && key0 < ctx) ? __ldg(bt + key0 / ps) : -1;
         };
-        auto issue = [&](bool is_k, int t, int row) -> bool {
-            const int nst = is_k ? KST : VST, st = t % nst;
-            const unsigned nbox = __popc(__ballot_sync(0xffffffffu, row >= 0));
-            bool ok = true;
-            // a K stage is free once S of the tile KST back is done, a V stage once
-            // PV of the tile VST back is done
-            if (t >= nst) {
-                const int prev = t - nst;
-                ok = wait_bar(is_k ? bars.s_done(prev % NSB) : bars.pv_done(prev % NSB), (prev / NSB) & 1,
-                              abort_flag, p.status);
-            }
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!ok) return false;
-            const uint32_t bar = is_k ? bars.k_full(st) : bars.v_full(st);
-            if (lane == 0) ptx::mbar_arrive_expect_tx(bar, nbox * 16 * 128);
-            __syncwarp();
-            if (row >= 0) {
-                const uint32_t dst = sbase + (is_k ? kSmemK : kSmemV) + st * kTile + my_half * kAtom + my_group * 2048;
-                ptx::tma_load_3d(dst, is_k ? &tm_k : &tm_v, bar, 64 * my_half, kvh, row);
-            }
-            return true;
-        };
-        int row_prev = -1;
-        for (int t = 0; t <= n_tiles; ++t) {
+        int pg = page_of(0);
+        int t = 0;
+        for (; t < n_tiles; ++t) {
+            const int pg_next = page_of(t + 1);
+            const int key0 = (t_first + t) * BN + 16 * group;
             int row = -1;
-            if (t < n_tiles) {
-                if (t > 0 && (t & 3) == 0) {
-                    pg_cur = pg_next;
-                    pg_next = load_pages(t / 4 + 1);
+            if (my_lane && key0 < ctx) {
+                if (pg < 0 || pg >= p.num_pages) {
+                    if (half == 0) record_error(p.status, PKV_ERR_DEVICE_RANGE, pg);
+                } else {
+                    row = pg * ps + key0 % ps;
                 }
-                row = row_of(t, pg_cur);
-                if (!issue(true, t, row)) break;
             }
-            if (t >= 1 && !issue(false, t - 1, row_prev)) break;
-            row_prev = row;
+            const int st = t % nst;
+            bool ok = true;
+            if (t >= nst) {
+                // a K stage is free once S of the last tile KST key tiles back is done,
+                // a V stage once PV of the last tile VST key tiles back is done
+                const int prev = t - nst;
+                ok = wait_bar(is_k ? bars.s_full(NT - 1, st) : bars.pv_done(st), (prev / nst) & 1, abort_flag,
+                              p.status);
+            }
+            if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) break;
+            const unsigned nbox = __popc(__ballot_sync(0xffffffffu, row >= 0));
+            const uint32_t full = is_k ? bars.k_full(st) : bars.v_full(st);
+            if (lane == 0) ptx::mbar_arrive_expect_tx(full, nbox * 16 * 128);
+            __syncwarp();
+            if (row >= 0)
+                ptx::tma_load_3d(ring + st * L::kTile + half * kAtom + group * 2048, map, full, 64 * half, kvh, row);
+            pg = pg_next;
+        }
+        if (*abort_flag && lane == 0) {
+            // let the copies this warp issued land before the CTA's shared memory is released
+            for (int u = max(0, t - nst); u < t; ++u)
+                ptx::mbar_wait(is_k ? bars.k_full(u % nst) : bars.v_full(u % nst), (u / nst) & 1, kSpinLimit >> 4);
+            if (is_k) ptx::mbar_wait(bars.q_full(), 0, kSpinLimit >> 4);
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------ MMA issuer ------------------------------
-        // S runs two tiles ahead of PV (S_0 S_1 | PV_0 S_2 | PV_1 S_3 | ...), so the
-        // softmax of tile i+1 never waits for P_i.  The ring slots are template
-        // arguments of the issue helpers and the TMEM base is 0, so every MMA
-        // operand is a constant.
         if (lane == 0) {
-            bool ok = wait_bar(bars.q_full(), 0, abort_flag, p.status);
-            auto issue_s = [&](int j) {
-                if (!wait_bar(bars.k_full(j % KST), (j / KST) & 1, abort_flag, p.status)) return false;
-                if (j >= NSB && !wait_bar(bars.pv_done(j % NSB), ((j / NSB) - 1) & 1, abort_flag, p.status))
-                    return false;
-                ptx::tc_fence_after();
-                switch (j % 3) {
-                    case 0: mma_s<T, 0>(sbase, bars); break;
-                    case 1: mma_s<T, 1>(sbase, bars); break;
-                    default: mma_s<T, 2>(sbase, bars); break;
-                }
-                return true;
-            };
-            auto issue_pv = [&](int i) {
-                if (!wait_bar(bars.p_full(i % NSB), (i / NSB) & 1, abort_flag, p.status)) return false;
-                if (!wait_bar(bars.v_full(i % VST), (i / VST) & 1, abort_flag, p.status)) return false;
-                ptx::tc_fence_after();
-                switch (i == 0 ? -1 : i % 6) {
-                    case -1: mma_pv<T, 0, 0, false>(sbase, bars); break;
-                    case 0: mma_pv<T, 0, 0, true>(sbase, bars); break;
-                    case 1: mma_pv<T, 1, 1, true>(sbase, bars); break;
-                    case 2: mma_pv<T, 2, 0, true>(sbase, bars); break;
-                    case 3: mma_pv<T, 0, 1, true>(sbase, bars); break;
-                    case 4: mma_pv<T, 1, 0, true>(sbase, bars); break;
-                    default: mma_pv<T, 2, 1, true>(sbase, bars); break;
-                }
-                return true;
-            };
-            ok = ok && issue_s(0) && (n_tiles < 2 || issue_s(1));
-            for (int i = 0; i < n_tiles && ok; ++i) {
-                ok = issue_pv(i);
-                if (ok && i + 2 < n_tiles) ok = issue_s(i + 2);
-            }
+            const Issuer<T, HD, NT> mma{sbase, bars, abort_flag, p.status};
+            mma.run(n_tiles);
             // drain: every tcgen05 op issued by this thread completes before TMEM is freed
             ptx::tc_commit(bars.mma_done());
             ptx::mbar_wait(bars.mma_done(), 0, kSpinLimit);
         }
+    }
     } else {
+    ptx_setmaxnreg_inc<216>();
+    if (warp < kSoftWarp0 + 4 * NT) {
         // ------------------------------ softmax + epilogue ------------------------------
-        // Warp w reaches TMEM lanes 32*(w%4)..+31 (its quarter of the rows); the two
-        // warps of a quarter split the 128 columns of S (and of O) into halves and
-        // exchange row maxima (and finally row sums) through shared memory.
-        const int quarter = warp & 3, hf = (warp - kSoftmaxWarp0) >> 2;
-        const int row = quarter * 32 + lane;                        // TMEM lane == tile row
-        const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-        const int c0 = hf * 64;                                     // this warp's S / O columns
-        float* red = reinterpret_cast<float*>(smem + kSmemRed);     // [2 bufs][2 halves][BM]
-        float* lsum = red + 2 * 2 * BM;                             // [2 halves][BM]
-        const int lim = min(p.causal ? ctx - n + r0 + row : ctx - 1, ctx - 1);
-        const int row_lo = w > 0 ? max(0, ctx - n + r0 + row - w + 1) : 0;     // this row's first key
+        const int x = (warp - kSoftWarp0) >> 2;                  // query tile (head h0 + x)
+        const int quarter = warp & 3;                            // TMEM lanes this warp reaches
+        const int row = quarter * 32 + lane;                     // TMEM lane == tile row
+        const uint32_t trow = static_cast<uint32_t>(quarter * 32) << 16;
+        const uint32_t tS = trow + x * 128, tO = trow + kOCol + x * 128;
+        const int pos = ctx - n + r0 + row;
+        const int lim = p.causal ? min(pos, ctx - 1) : ctx - 1;
+        const int row_lo = w > 0 ? max(0, pos - w + 1) : 0;      // this row's first key
         const float sl2 = p.scale_log2;
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < n_tiles; ++j) {
-            const int bj = j % NSB;
-            ok = wait_bar(bars.s_done(bj), (j / NSB) & 1, abort_flag, p.status);
+            ok = wait_bar(bars.s_full(x, j % KST), (j / KST) & 1, abort_flag, p.status);
             if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
             ptx::tc_fence_after();
-            uint32_t r[64];
-            {
-                uint32_t (&r0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[0]);
-                uint32_t (&r1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[32]);
-                ptx::tmem_ld32(trow + bj * 128 + c0, r0);
-                ptx::tmem_ld32(trow + bj * 128 + c0 + 32, r1);
-            }
-            ptx::tc_wait_ld();
-            float x[64];
+            uint32_t r[128];
 #pragma unroll
-            for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(r[c]);
-            const int jt = tile_of(j);
+            for (int c = 0; c < 4; ++c) ptx::tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+            ptx::tc_wait_ld();
+            float v[128];
+#pragma unroll
+            for (int c = 0; c < 128; ++c) v[c] = __uint_as_float(r[c]);
+            const int jt = t_first + j;
             if (jt * BN + BN - 1 > min_lim || jt * BN < lo_mask) {  // diagonal / last / window edge
 #pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    const int key = jt * BN + c0 + c;
-                    if (key > lim || key < row_lo) x[c] = -INFINITY;
+                for (int c = 0; c < 128; ++c) {
+                    const int key = jt * BN + c;
+                    if (key > lim || key < row_lo) v[c] = -INFINITY;
                 }
             }
-            float mh = x[0];
+            float m4[4] = {v[0], v[1], v[2], v[3]};
 #pragma unroll
-            for (int c = 1; c < 64; ++c) mh = fmaxf(mh, x[c]);
-            float* rb = red + (j & 1) * 2 * BM;
-            rb[hf * BM + row] = mh;
-            named_bar_sync(1 + quarter, 64);
+            for (int c = 4; c < 128; ++c) m4[c & 3] = fmaxf(m4[c & 3], v[c]);
             // -inf only for a row that sees no key of this tile (possible with a window)
-            const float mt = fmaxf(mh, rb[(1 - hf) * BM + row]) * sl2;
+            const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
             if (j == 0) {
                 m_ref = mt;
             } else if (__any_sync(0xffffffffu, mt > m_ref + kRescaleThreshold)) {
+                // S_X(j) completed after PV_X(j-1) (same issuer, in order), so O_X is settled
                 const float m_new = fmaxf(m_ref, mt);
-                const float corr = ptx::ex2(m_ref - m_new);
+                const float corr = m_new == -INFINITY ? 1.f : ptx::ex2(m_ref - m_new);
                 l *= corr;
                 m_ref = m_new;
-                const int pj = j - 1;
-                ok = wait_bar(bars.pv_done(pj % NSB), (pj / NSB) & 1, abort_flag, p.status);
-                if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
-                ptx::tc_fence_after();
-#pragma unroll
-                for (int c32 = 0; c32 < 2; ++c32) {
-                    uint32_t o[32];
-                    ptx::tmem_ld32(trow + kOCol + c0 + c32 * 32, o);
+#pragma unroll 1
+                for (int c = 0; c < HD / 16; ++c) {              // 16 columns at a time: S is still live
+                    uint32_t o[16];
+                    tmem_ld16(tO + 16 * c, o);
                     ptx::tc_wait_ld();
-                    uint32_t w0[16], w1[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        w0[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
-                        w1[i] = __float_as_uint(__uint_as_float(o[16 + i]) * corr);
-                    }
-                    ptx::tmem_st16(trow + kOCol + c0 + c32 * 32, w0);
-                    ptx::tmem_st16(trow + kOCol + c0 + c32 * 32 + 16, w1);
+                    for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
+                    ptx::tmem_st16(tO + 16 * c, o);
                 }
-                ptx::tc_wait_st();
             }
             const float neg = m_ref == -INFINITY ? 0.f : -m_ref;      // no key seen yet: all p are 0
-            float rs = 0.f;
+            float rs[2] = {0.f, 0.f};
 #pragma unroll
-            for (int c16 = 0; c16 < 2; ++c16) {
-                uint32_t pk[16];
+            for (int c32 = 0; c32 < 2; ++c32) {
+                uint32_t pk[32];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int c = c16 * 32 + 2 * i;
-                    const float ya = fmaf(x[c], sl2, neg), yb = fmaf(x[c + 1], sl2, neg);
-                    const float a = ptx::ex2(ya), bb = ptx::ex2(yb);
-                    rs += a + bb;
+                for (int i = 0; i < 32; ++i) {
+                    const int c = c32 * 64 + 2 * i;
+                    const float a = ptx::ex2(fmaf(v[c], sl2, neg)), bb = ptx::ex2(fmaf(v[c + 1], sl2, neg));
+                    rs[i & 1] += a + bb;
                     pk[i] = pack2<T>(a, bb);
                 }
-                ptx::tmem_st16(trow + bj * 128 + hf * 32 + c16 * 16, pk);
+                tmem_st32(tS + 32 * c32, pk);                   // P column c holds keys 2c, 2c+1
             }
-            l += rs;
+            l += rs[0] + rs[1];
             ptx::tc_wait_st();
-            if (ctx < (jt + 1) * BN) {
+            if (x == 0 && ctx < (jt + 1) * BN) {
                 // V rows past the context (tail of the last page, or never loaded) must be
-                // finite zeros: P is 0 there but 0 * NaN would poison O.
+                // finite zeros: P is 0 there but 0 * NaN would poison O.  Tile A's warps do it
+                // before PV_A(j), which runs before PV_B(j).
                 const int vs = j % VST;
                 ok = wait_bar(bars.v_full(vs), (j / VST) & 1, abort_flag, p.status);
                 if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
                 const int first = ctx - jt * BN;                    // first invalid row of the tile
-                uint4* vt = reinterpret_cast<uint4*>(smem + kSmemV + vs * kTile);
-                const int tid = threadIdx.x - kSoftmaxWarp0 * 32;
-                for (int idx = tid; idx < 2 * (BN - first) * 8; idx += kSoftmaxWarps * 32) {
-                    const int half = idx / ((BN - first) * 8), rem = idx % ((BN - first) * 8);
-                    vt[(half * kAtom + (first + rem / 8) * 128) / 16 + rem % 8] = make_uint4(0, 0, 0, 0);
+                uint4* vt = reinterpret_cast<uint4*>(smem + L::kV + vs * L::kTile);
+                const int tid = threadIdx.x - kSoftWarp0 * 32, per = (BN - first) * 8;
+                for (int idx = tid; idx < L::NH * per; idx += 128) {
+                    const int a = idx / per, rem = idx % per;
+                    vt[(a * kAtom + (first + rem / 8) * 128) / 16 + rem % 8] = make_uint4(0, 0, 0, 0);
                 }
                 ptx::fence_proxy_async_smem();
             }
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(bars.p_full(bj));      // one arrival per warp
+            if (lane == 0) ptx::mbar_arrive(bars.p_full(x));       // one arrival per warp
         }
-        // epilogue: O / l -> out (each warp writes its 64 output columns)
-        if (ok) {
-            const int pj = n_tiles - 1;
-            ok = wait_bar(bars.pv_done(pj % NSB), (pj / NSB) & 1, abort_flag, p.status);
-        }
-        lsum[hf * BM + row] = l;
-        named_bar_sync(1 + quarter, 64);
+        // epilogue: O / l -> out
+        if (ok) ok = wait_bar(bars.o_full(x), 0, abort_flag, p.status);
         if (__all_sync(0xffffffffu, ok)) {
             ptx::tc_fence_after();
-            const float inv = 1.f / (l + lsum[(1 - hf) * BM + row]);
+            const float inv = 1.f / l;
             const bool store = r0 + row < n;
-            T* out = static_cast<T*>(p.out) + (static_cast<size_t>(q0 + r0 + row) * Hq + h) * HD + c0;
+            T* out = static_cast<T*>(p.out) + (static_cast<size_t>(q0 + r0 + row) * Hq + h0 + x) * HD;
 #pragma unroll
-            for (int c32 = 0; c32 < 2; ++c32) {
+            for (int c = 0; c < HD / 32; ++c) {
                 uint32_t o[32];
-                ptx::tmem_ld32(trow + kOCol + c0 + c32 * 32, o);
+                ptx::tmem_ld32(tO + 32 * c, o);
                 ptx::tc_wait_ld();
-                uint32_t w[16];
+                uint32_t wv[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
-                    w[i] = pack2<T>(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+                    wv[i] = pack2<T>(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
                 if (store) {
-                    uint4* dst = reinterpret_cast<uint4*>(out + c32 * 32);
+                    uint4* dst = reinterpret_cast<uint4*>(out + 32 * c);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
                 }
             }
         }
     }
 
+    }
+
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == 0 && lane == 0 && *abort_flag) {
-        // let in-flight TMA writes land before the shared memory is handed to another CTA
-        for (int t = 0; t < KST; ++t) ptx::mbar_wait(bars.k_full(t), 0, kSpinLimit >> 4);
-    }
     if (warp == kMmaWarp) {
+        __syncwarp();
         ptx::tc_fence_after();
         ptx::tmem_dealloc(*tmem_slot, kTmemCols);
     }
@@ -511,13 +559,13 @@ EncodeTiled encoder() {
     return fn;
 }
 
-// 3-D map over a [rows][heads][128] tensor of 16-bit elements, box {64, 1, box_rows}, SW128.
-bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t heads, uint64_t rows,
+// 3-D map over a [rows][heads][hd] tensor of 16-bit elements, box {64, 1, box_rows}, SW128.
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t hd, uint64_t heads, uint64_t rows,
               uint32_t box_rows) {
     EncodeTiled enc = encoder();
     if (!enc) return false;
-    const cuuint64_t dims[3] = {HD, heads, rows};
-    const cuuint64_t strides[2] = {HD * 2, heads * HD * 2};
+    const cuuint64_t dims[3] = {hd, heads, rows};
+    const cuuint64_t strides[2] = {hd * 2, heads * hd * 2};
     const cuuint32_t box[3] = {64, 1, box_rows};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -525,21 +573,33 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename T>
+template <typename T, int HD, int NT>
 cudaError_t run(const PrefillParams& p, cudaStream_t stream) {
+    using L = Layout<HD, NT>;
     const CUtensorMapDataType dt =
         std::is_same<T, __nv_bfloat16>::value ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     CUtensorMap tq, tk, tv;
     const uint64_t pool_rows = static_cast<uint64_t>(p.num_pages) * p.page_size;
-    if (!make_map(&tq, p.q, dt, p.num_q_heads, p.total_q, BM) ||
-        !make_map(&tk, p.k_pages, dt, p.num_kv_heads, pool_rows, 16) ||
-        !make_map(&tv, p.v_pages, dt, p.num_kv_heads, pool_rows, 16))
+    if (!make_map(&tq, p.q, dt, HD, p.num_q_heads, p.total_q, BM) ||
+        !make_map(&tk, p.k_pages, dt, HD, p.num_kv_heads, pool_rows, 16) ||
+        !make_map(&tv, p.v_pages, dt, HD, p.num_kv_heads, pool_rows, 16))
         return cudaErrorInvalidValue;
-    dim3 grid(p.num_q_heads, p.num_seqs, ceil_div(p.max_q_len, BM));
-    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(prefill_tc_kernel<T>), kSmemBytes);
+    dim3 grid(p.num_q_heads / NT, p.num_seqs, ceil_div(p.max_q_len, BM));
+    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(prefill_tc_kernel<T, HD, NT>), L::kSmem);
     if (e != cudaSuccess) return e;
-    prefill_tc_kernel<T><<<grid, kThreads, kSmemBytes, stream>>>(p, tq, tk, tv);
+    prefill_tc_kernel<T, HD, NT><<<grid, kThreads, L::kSmem, stream>>>(p, tq, tk, tv);
     return cudaGetLastError();
+}
+
+template <typename T, int HD>
+cudaError_t run_hd(const PrefillParams& p, cudaStream_t stream) {
+    // pair the heads of a group when the group size is even
+    return (p.num_q_heads / p.num_kv_heads) % 2 == 0 ? run<T, HD, 2>(p, stream) : run<T, HD, 1>(p, stream);
+}
+
+template <typename T>
+cudaError_t run_t(const PrefillParams& p, cudaStream_t stream) {
+    return p.head_dim == 64 ? run_hd<T, 64>(p, stream) : run_hd<T, 128>(p, stream);
 }
 
 }  // namespace
@@ -569,7 +629,7 @@ cudaError_t launch_wait_timeout_selftest(DeviceStatus* st, cudaStream_t stream) 
 
 cudaError_t launch_prefill(const PrefillParams& p, pkv_dtype dtype, cudaStream_t stream) {
     if (p.max_q_len <= 0 || p.num_seqs <= 0 || p.total_q <= 0) return cudaSuccess;
-    return dtype == PKV_BF16 ? run<__nv_bfloat16>(p, stream) : run<__half>(p, stream);
+    return dtype == PKV_BF16 ? run_t<__nv_bfloat16>(p, stream) : run_t<__half>(p, stream);
 }
 
 }  // namespace pkv

@@ -98,10 +98,14 @@ def test_host_validation_rejects_before_launch(lib):
     rc = lib.pkv_paged_attention_decode(fake, fake, fake, fake, fake, 1.0, fake, 2, 8, 2, 128, 16, 1024,
                                         10, 1, 1, None, None, None, 0, 0, None)
     assert rc == -3
-    # prefill: head_dim 64 unsupported, fp32 unsupported
+    # prefill: head_dim 96 unsupported (64 and 128 are), fp32 unsupported, scale must be > 0
     rc = lib.pkv_paged_attention_prefill(fake, fake, fake, fake, fake, fake, 1, 1.0, fake, 2, 8, 4, 8, 2,
-                                         64, 16, 4, 10, 1, None)
+                                         96, 16, 4, 10, 1, None)
     assert rc == -2
+    for bad_scale in (0.0, -0.5):
+        rc = lib.pkv_paged_attention_prefill(fake, fake, fake, fake, fake, fake, 1, bad_scale, fake, 2, 8, 4, 8,
+                                             2, 128, 16, 4, 10, 1, None)
+        assert rc == -1
     rc = lib.pkv_paged_attention_prefill(fake, fake, fake, fake, fake, fake, 1, 1.0, fake, 2, 8, 4, 8, 2,
                                          128, 16, 4, 10, 0, None)
     assert rc == -2

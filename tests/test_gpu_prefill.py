@@ -33,9 +33,9 @@ def run_prefill(case, causal=True, items=None, tol=2e-2, window=0):
     assert_close(got, want, tol, case.name)
 
 
-def case(idx, chunks, private_prefix=0, shared_prefix=32, Hq=8, Hkv=2, ps=16, dtype="bf16"):
+def case(idx, chunks, private_prefix=0, shared_prefix=32, Hq=8, Hkv=2, ps=16, dtype="bf16", D=128):
     return W.prefill_case(name=f"prefill{idx}", config_index=200 + idx, num_seqs=len(chunks),
-                          num_q_heads=Hq, num_kv_heads=Hkv, head_dim=128, page_size=ps, dtype=dtype,
+                          num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D, page_size=ps, dtype=dtype,
                           shared_prefix=shared_prefix, chunk_lens=np.array(chunks),
                           private_prefix=private_prefix)
 
@@ -107,3 +107,27 @@ def test_many_ragged_sequences():
     # 40 sequences, seeded chunk lengths 0..149 (some empty), one shared prefix
     chunks = np.random.default_rng(7).integers(0, 150, 40)
     run_prefill(case(13, chunks=tuple(int(c) for c in chunks), private_prefix=3, shared_prefix=48))
+
+
+# ---- head_dim 64, and query-head groups that cannot be paired ----------------------
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_head_dim_64(causal):
+    # ragged chunks after a shared and a private prefix, chunks starting mid-page
+    run_prefill(case(30, chunks=(1, 5, 64, 130, 200, 128), private_prefix=7, D=64), causal=causal)
+
+
+@pytest.mark.parametrize("window", [1, 100, 129])
+def test_head_dim_64_sliding_window(window):
+    run_prefill(case(31, chunks=(3, 140, 77), private_prefix=5, shared_prefix=256, D=64), window=window)
+
+
+def test_head_dim_64_fp16_large_pages():
+    run_prefill(case(32, chunks=(90, 257), Hq=4, Hkv=4, ps=256, shared_prefix=256, private_prefix=3, D=64,
+                     dtype="f16"))
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(6, 2), (3, 1)])
+def test_odd_group_sizes(Hq, Hkv):
+    # groups of 3 query heads: one query tile per CTA instead of a pair
+    run_prefill(case(33 + Hq, chunks=(17, 130, 256), Hq=Hq, Hkv=Hkv, private_prefix=9))
