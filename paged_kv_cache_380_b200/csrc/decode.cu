@@ -97,9 +97,9 @@ decode_mma_kernel(const DecodeParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
-    // partitions vary slowest: every sequence's first (longest) partitions are
-    // dispatched before the partial remainders, which then fill the tail
-    const int kvh = blockIdx.x, b = blockIdx.y, split = blockIdx.z;
+    // KV heads vary fastest: the CTAs of one token range for all KV heads run side by
+    // side, so a token's K/V rows (all heads contiguous in the page) are read together
+    const int kvh = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
     const int Hq = p.num_q_heads, Hkv = p.num_kv_heads, G = Hq / Hkv, ps = p.page_size;
 
     const int ctx = __ldg(p.context_lens + b);
@@ -554,7 +554,7 @@ cudaError_t run_mma(const DecodeParams& p, cudaStream_t stream) {
     auto kern = decode_mma_kernel<QT, KVT, HD, NT, kWarps, kStages>;
     cudaError_t e0 = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), Cfg::kSmem);
     if (e0 != cudaSuccess) return e0;
-    dim3 grid(p.num_kv_heads, p.num_seqs, p.max_splits);
+    dim3 grid(p.num_kv_heads, p.max_splits, p.num_seqs);
     kern<<<grid, kWarps * 32, Cfg::kSmem, stream>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || p.max_splits == 1) return e;

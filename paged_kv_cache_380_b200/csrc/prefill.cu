@@ -57,7 +57,6 @@ namespace {
 
 constexpr int BM = 128, BN = 128;               // query rows / keys per tile
 constexpr int KST = 3, VST = 2;                 // K stages, V stages
-constexpr int kRing = 6;                        // KST and VST ring positions repeat every 6 key tiles
 constexpr int kKWarp = 0, kVWarp = 1, kMmaWarp = 2, kSoftWarp0 = 4;
 constexpr int kThreads = 12 * 32;               // 3 warpgroups
 constexpr uint32_t kTmemCols = 512;
@@ -87,8 +86,8 @@ struct Bars {
     uint32_t base;
     __device__ __forceinline__ uint32_t at(int i) const { return base + 8 * i; }
     __device__ __forceinline__ uint32_t q_full() const { return at(0); }
-    __device__ __forceinline__ uint32_t k_full(int s) const { return at(1 + s); }
-    __device__ __forceinline__ uint32_t v_full(int s) const { return at(1 + KST + s); }
+    // load step t (slot t % KST): K tile t and V tile t-1 landed (one arrival from each producer warp)
+    __device__ __forceinline__ uint32_t kv_full(int s) const { return at(1 + s); }
     // S_X(j) done (and, for the last tile, K stage s free), one barrier per K stage
     __device__ __forceinline__ uint32_t s_full(int x, int s) const { return at(1 + KST + VST + x * KST + s); }
     __device__ __forceinline__ uint32_t p_full(int x) const { return at(1 + 3 * KST + VST + x); }
@@ -137,14 +136,69 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         : "r"(taddr));
 }
 
-// Per-warpgroup register budget changes (all threads of a warpgroup execute them).
-template <int N>
-__device__ __forceinline__ void ptx_setmaxnreg_dec() {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N));
+// Orders the uses of registers written by a tcgen05.ld after the tcgen05.wait::ld
+// that precedes this call (the compiler sees the registers as rewritten here).
+__device__ __forceinline__ void reg_fence32(uint32_t* r) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                   "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                   "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
 }
-template <int N>
-__device__ __forceinline__ void ptx_setmaxnreg_inc() {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N));
+
+// 64 consecutive fp32 columns of this thread's TMEM lane into v (waits for the load).
+__device__ __forceinline__ void load_half(uint32_t taddr, float (&v)[64]) {
+    uint32_t r[64];
+    ptx::tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+    ptx::tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+    ptx::tc_wait_ld();
+    reg_fence32(&r[0]);
+    reg_fence32(&r[32]);
+#pragma unroll
+    for (int c = 0; c < 64; ++c) v[c] = __uint_as_float(r[c]);
+}
+// Scores of keys outside lo .. lim (key of column c is key0 + c) become -inf.
+__device__ __forceinline__ void mask_half(float (&v)[64], int key0, int lim, int lo) {
+#pragma unroll
+    for (int c = 0; c < 64; ++c)
+        if (key0 + c > lim || key0 + c < lo) v[c] = -INFINITY;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// Two lanes of packed fp32 arithmetic (one instruction for both).
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// 2^y for the two lanes of y in fp32 on the SFU (which evaluates 4 exponentials per
+// clock per sub-partition whatever their width, so a packed bf16 form saves no SFU
+// time), both added to sum; returns the pair rounded to T and packed (low half =
+// first lane).
+template <typename T>
+__device__ __forceinline__ uint32_t exp2_pair(uint64_t y, uint64_t& sum) {
+    float y0, y1;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(y0), "=f"(y1) : "l"(y));
+    const float e0 = ptx::ex2(y0), e1 = ptx::ex2(y1);
+    sum = fadd2(sum, f2pack(e0, e1));
+    return pack2<T>(e0, e1);
 }
 
 #ifndef PKV_PREFILL_MMA_SLEEP
@@ -173,13 +227,25 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     return false;
 }
 
-// The MMA issuer's view of the CTA: operand addresses are compile-time offsets
-// from the shared-memory base, and the ring slots are template arguments, so
-// every MMA operand is a constant.
+// Every lane of the warp waits (measured faster than one polling lane and a
+// broadcast); the result is made warp-uniform.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int lane, volatile int* abort_flag,
+                                          DeviceStatus* st) {
+    (void)lane;
+    const bool ok = wait_bar(bar, parity, abort_flag, st);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// The MMA issuer.  One code path serves every ring slot: a slot only moves the
+// shared-memory start address, i.e. adds a constant to the low word of the
+// descriptor (the address field holds addr >> 4 in 14 bits, and shared memory
+// ends below 256 KB, so the sum never carries out of it).  One compact loop keeps
+// the issuing thread's instruction stream small.
 template <typename T, int HD, int NT>
 struct Issuer {
     using L = Layout<HD, NT>;
-    uint32_t sbase;
+    uint64_t dq[NT];                 // Q of each tile
+    uint64_t dk, dv;                 // K and V stage 0
     Bars bars;
     volatile int* abort_flag;
     DeviceStatus* status;
@@ -187,81 +253,58 @@ struct Issuer {
     __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity) const {
         return wait_bar<PKV_PREFILL_MMA_SLEEP != 0>(bar, parity, abort_flag, status);
     }
-    // The shared-memory base, opaque to the compiler: descriptors are rebuilt at
-    // each use (a few integer instructions) instead of being hoisted out of the
-    // key loop into dozens of live registers.
-    __device__ __forceinline__ uint32_t base() const {
-        uint32_t b;
-        asm volatile("mov.b32 %0, %1;\n" : "=r"(b) : "r"(sbase));
-        return b;
-    }
-    // S_X = Q_X K[stage KS]^T, then one commit: "S_X done" (+ K stage free for the last tile).
-    template <int X, int KS>
-    __device__ __forceinline__ void s() const {
+    // S_x = Q_x K[stage ks]^T, then one commit: "S_x done" (+ K stage free for the last tile).
+    __device__ __forceinline__ void s(int x, int ks) const {
         constexpr uint32_t id = idesc_f16<T>(BM, BN, 0);
-        const uint32_t sb = base();
-        const uint32_t qa = sb + L::kQ + X * L::kTile, ka = sb + L::kK + KS * L::kTile;
+        const uint64_t a = dq[x], b = dk + static_cast<uint64_t>((ks * L::kTile) >> 4);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
-            ptx::tc_mma_ss(X * 128, sdesc(qa + off, 16, 1024), sdesc(ka + off, 16, 1024), id, kk > 0 ? 1u : 0u);
+            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kAtom + (kk & 3) * 32) >> 4);
+            ptx::tc_mma_ss(static_cast<uint32_t>(x * 128), a + off, b + off, id, kk > 0 ? 1u : 0u);
         }
-        ptx::tc_commit(bars.s_full(X, KS));
+        ptx::tc_commit(bars.s_full(x, ks));
     }
-    // O_X (+)= P_X V[stage VS]; the first key tile overwrites O.
-    template <int X, int VS>
-    __device__ __forceinline__ void pv(bool acc) const {
+    // O_x (+)= P_x V[stage vs]; the first key tile overwrites O.
+    __device__ __forceinline__ void pv(int x, int vs, bool acc) const {
         constexpr uint32_t id = idesc_f16<T>(BM, HD, 1);
-        const uint32_t va = base() + L::kV + VS * L::kTile;
+        const uint64_t b = dv + static_cast<uint64_t>((vs * L::kTile) >> 4);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-            ptx::tc_mma_ts(kOCol + X * 128, X * 128 + kk * 8, sdesc(va + kk * 2048, kAtom, 1024), id,
-                           (acc || kk > 0) ? 1u : 0u);
+            ptx::tc_mma_ts(kOCol + x * 128, static_cast<uint32_t>(x * 128 + kk * 8), b + static_cast<uint64_t>((kk * 2048) >> 4),
+                           id, (acc || kk > 0) ? 1u : 0u);
     }
-    // Key tile j (R = j % kRing): PV_A(j) S_A(j+1) [PV_B(j) S_B(j+1)].
-    template <int R>
-    __device__ __forceinline__ bool step(int j, int n) const {
-        constexpr int VS = R % VST, KS1 = (R + 1) % KST;
-        const bool more = j + 1 < n;
-        if (!wait(bars.p_full(0), j & 1) || !wait(bars.v_full(VS), (j / VST) & 1)) return false;
-        ptx::tc_fence_after();
-        pv<0, VS>(j > 0);
-        if constexpr (NT == 1) ptx::tc_commit(bars.pv_done(VS));
-        if (!more) ptx::tc_commit(bars.o_full(0));
-        if (more) {
-            if (!wait(bars.k_full(KS1), ((j + 1) / KST) & 1)) return false;
-            ptx::tc_fence_after();
-            s<0, KS1>();
-        }
-        if constexpr (NT == 2) {
-            if (!wait(bars.p_full(1), j & 1)) return false;
-            ptx::tc_fence_after();
-            pv<1, VS>(j > 0);
-            ptx::tc_commit(bars.pv_done(VS));
-            if (!more) ptx::tc_commit(bars.o_full(1));
-            if (more) s<1, KS1>();
-        }
-        return true;
-    }
+    // Key tile j: PV_A(j) S_A(j+1) [PV_B(j) S_B(j+1)].  Three barrier probes per key tile
+    // (P_A, the K/V step, P_B): each probe costs the tensor pipe about as much as three
+    // MMAs, so there are no others.
     __device__ void run(int n) const {
-        if (!wait(bars.q_full(), 0) || !wait(bars.k_full(0), 0)) return;
+        if (!wait(bars.q_full(), 0) || !wait(bars.kv_full(0), 0)) return;
         ptx::tc_fence_after();
-        s<0, 0>();
-        if constexpr (NT == 2) s<1, 0>();
-        bool ok = true;
-        for (int j = 0; j < n && ok; ++j) {
-            switch (j % kRing) {
-            case 0: ok = step<0>(j, n); break;
-            case 1: ok = step<1>(j, n); break;
-            case 2: ok = step<2>(j, n); break;
-            case 3: ok = step<3>(j, n); break;
-            case 4: ok = step<4>(j, n); break;
-            default: ok = step<5>(j, n); break;
+        for (int x = 0; x < NT; ++x) s(x, 0);
+        int vs = 0, ks = 0;                                      // j % VST, j % KST
+        for (int j = 0; j < n; ++j) {
+            const int ks1 = ks + 1 == KST ? 0 : ks + 1;
+            const bool more = j + 1 < n;
+            // load step j+1 holds V tile j (for PV) and K tile j+1 (for the next S)
+            if (!wait(bars.p_full(0), j & 1) || !wait(bars.kv_full(ks1), ((j + 1) / KST) & 1)) return;
+            ptx::tc_fence_after();
+            pv(0, vs, j > 0);
+            if (NT == 1) ptx::tc_commit(bars.pv_done(vs));
+            if (!more) ptx::tc_commit(bars.o_full(0));
+            if (more) s(0, ks1);
+            if (NT == 2) {
+                if (!wait(bars.p_full(1), j & 1)) return;
+                ptx::tc_fence_after();
+                pv(1, vs, j > 0);
+                ptx::tc_commit(bars.pv_done(vs));
+                if (!more) ptx::tc_commit(bars.o_full(1));
+                if (more) s(1, ks1);
             }
+            static_assert(VST == 2, "V ring of two stages");
+            vs ^= 1;
+            ks = ks1;
         }
     }
 };
-
 template <typename T, int HD, int NT>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
@@ -303,13 +346,10 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
     if (threadIdx.x == 0) {
         ptx::mbar_init(bars.q_full(), 1);
         for (int i = 0; i < KST; ++i) {
-            ptx::mbar_init(bars.k_full(i), 1);
+            ptx::mbar_init(bars.kv_full(i), 2);
             for (int x = 0; x < 2; ++x) ptx::mbar_init(bars.s_full(x, i), 1);
         }
-        for (int i = 0; i < VST; ++i) {
-            ptx::mbar_init(bars.v_full(i), 1);
-            ptx::mbar_init(bars.pv_done(i), 1);
-        }
+        for (int i = 0; i < VST; ++i) ptx::mbar_init(bars.pv_done(i), 1);
         for (int x = 0; x < 2; ++x) {
             ptx::mbar_init(bars.p_full(x), 4);                  // one arrival per softmax warp
             ptx::mbar_init(bars.o_full(x), 1);
@@ -332,12 +372,6 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
         record_error(p.status, PKV_ERR_CUDA, static_cast<long long>(*tmem_slot));
     }
 
-    // Register split (setmaxnreg acts per warpgroup): the producer / MMA warpgroup
-    // gives registers back so that each softmax thread can hold a whole S row.
-    // Launch: 384 threads x 168; after: 128 x 56 + 256 x 216 = 62464 <= 64512.
-    __syncwarp();
-    if (warp < 4) {
-    ptx_setmaxnreg_dec<56>();
     if (warp == kKWarp || warp == kVWarp) {
         // ------------------------------ TMA producers ------------------------------
         // A key tile is 8 page groups of 16 rows x NH column atoms: one box per lane.
@@ -360,16 +394,26 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
         const int group = lane / L::NH, half = lane % L::NH;
         const bool my_lane = group < 8;
         const int32_t* bt = p.block_tables + static_cast<size_t>(b) * p.max_pages_per_seq;
-        // physical page of my group in tile t (read one tile ahead of its use), or -1
-        auto page_of = [&](int t) -> int {
-            const int key0 = (t_first + t) * BN + 16 * group;
-            return (my_lane && t < n_tiles && key0 < ctx) ? __ldg(bt + key0 / ps) : -1;
+        // Load step t: the K warp loads K tile t, the V warp V tile t-1 (V runs one tile
+        // behind K), both onto kv_full(t % KST); a warp with no tile at this step just
+        // arrives.  Page indices are read one tile ahead of their use.
+        const int lag = is_k ? 0 : 1;
+        auto page_of = [&](int u) -> int {
+            const int key0 = (t_first + u) * BN + 16 * group;
+            return (my_lane && u >= 0 && u < n_tiles && key0 < ctx) ? __ldg(bt + key0 / ps) : -1;
         };
-        int pg = page_of(0);
+        int pg = page_of(-lag);
         int t = 0;
-        for (; t < n_tiles; ++t) {
-            const int pg_next = page_of(t + 1);
-            const int key0 = (t_first + t) * BN + 16 * group;
+        for (; t <= n_tiles; ++t) {
+            const int u = t - lag;                                  // tile this warp loads at step t
+            const int pg_next = page_of(u + 1);
+            const uint32_t full = bars.kv_full(t % KST);
+            if (u < 0 || u >= n_tiles) {
+                if (lane == 0) ptx::mbar_arrive(full);
+                pg = pg_next;
+                continue;
+            }
+            const int key0 = (t_first + u) * BN + 16 * group;
             int row = -1;
             if (my_lane && key0 < ctx) {
                 if (pg < 0 || pg >= p.num_pages) {
@@ -378,18 +422,17 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
                     row = pg * ps + key0 % ps;
                 }
             }
-            const int st = t % nst;
+            const int st = u % nst;
             bool ok = true;
-            if (t >= nst) {
+            if (u >= nst) {
                 // a K stage is free once S of the last tile KST key tiles back is done,
                 // a V stage once PV of the last tile VST key tiles back is done
-                const int prev = t - nst;
-                ok = wait_bar(is_k ? bars.s_full(NT - 1, st) : bars.pv_done(st), (prev / nst) & 1, abort_flag,
-                              p.status);
+                const int prev = u - nst;
+                ok = warp_wait(is_k ? bars.s_full(NT - 1, st) : bars.pv_done(st), (prev / nst) & 1, lane, abort_flag,
+                               p.status);
             }
-            if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) break;
+            if (!ok) break;
             const unsigned nbox = __popc(__ballot_sync(0xffffffffu, row >= 0));
-            const uint32_t full = is_k ? bars.k_full(st) : bars.v_full(st);
             if (lane == 0) ptx::mbar_arrive_expect_tx(full, nbox * 16 * 128);
             __syncwarp();
             if (row >= 0)
@@ -398,23 +441,25 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
         }
         if (*abort_flag && lane == 0) {
             // let the copies this warp issued land before the CTA's shared memory is released
-            for (int u = max(0, t - nst); u < t; ++u)
-                ptx::mbar_wait(is_k ? bars.k_full(u % nst) : bars.v_full(u % nst), (u / nst) & 1, kSpinLimit >> 4);
+            for (int v = max(0, t - KST); v < t; ++v) ptx::mbar_wait(bars.kv_full(v % KST), (v / KST) & 1, kSpinLimit >> 4);
             if (is_k) ptx::mbar_wait(bars.q_full(), 0, kSpinLimit >> 4);
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------ MMA issuer ------------------------------
         if (lane == 0) {
-            const Issuer<T, HD, NT> mma{sbase, bars, abort_flag, p.status};
+            Issuer<T, HD, NT> mma;
+            for (int x = 0; x < NT; ++x) mma.dq[x] = sdesc(sbase + L::kQ + x * L::kTile, 16, 1024);
+            mma.dk = sdesc(sbase + L::kK, 16, 1024);
+            mma.dv = sdesc(sbase + L::kV, kAtom, 1024);
+            mma.bars = bars;
+            mma.abort_flag = abort_flag;
+            mma.status = p.status;
             mma.run(n_tiles);
             // drain: every tcgen05 op issued by this thread completes before TMEM is freed
             ptx::tc_commit(bars.mma_done());
             ptx::mbar_wait(bars.mma_done(), 0, kSpinLimit);
         }
-    }
-    } else {
-    ptx_setmaxnreg_inc<216>();
-    if (warp < kSoftWarp0 + 4 * NT) {
+    } else if (warp >= kSoftWarp0 && warp < kSoftWarp0 + 4 * NT) {
         // ------------------------------ softmax + epilogue ------------------------------
         const int x = (warp - kSoftWarp0) >> 2;                  // query tile (head h0 + x)
         const int quarter = warp & 3;                            // TMEM lanes this warp reaches
@@ -428,29 +473,29 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < n_tiles; ++j) {
-            ok = wait_bar(bars.s_full(x, j % KST), (j / KST) & 1, abort_flag, p.status);
-            if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+            ok = warp_wait(bars.s_full(x, j % KST), (j / KST) & 1, lane, abort_flag, p.status);
+            if (!ok) break;
             ptx::tc_fence_after();
-            uint32_t r[128];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) ptx::tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
-            ptx::tc_wait_ld();
-            float v[128];
-#pragma unroll
-            for (int c = 0; c < 128; ++c) v[c] = __uint_as_float(r[c]);
+            // Two passes over the row in 64-column halves (one compact loop body each; S
+            // is read from TMEM twice, which costs a few dozen cycles): the row max, then
+            // P = 2^(s * scale - m) written back over the first half of the S columns.
             const int jt = t_first + j;
-            if (jt * BN + BN - 1 > min_lim || jt * BN < lo_mask) {  // diagonal / last / window edge
+            const bool masked = jt * BN + BN - 1 > min_lim || jt * BN < lo_mask;   // diagonal / last / window edge
+            float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+            for (int hh = 0; hh < 2; ++hh) {
+                float v[64];
+                load_half(tS + 64 * hh, v);
+                if (masked) mask_half(v, jt * BN + 64 * hh, lim, row_lo);
+                // four independent max chains keep the reduction's latency short
 #pragma unroll
-                for (int c = 0; c < 128; ++c) {
-                    const int key = jt * BN + c;
-                    if (key > lim || key < row_lo) v[c] = -INFINITY;
+                for (int c = 0; c < 64; c += 8) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) mc[k] = max3(mc[k], v[c + 2 * k], v[c + 2 * k + 1]);
                 }
             }
-            float m4[4] = {v[0], v[1], v[2], v[3]};
-#pragma unroll
-            for (int c = 4; c < 128; ++c) m4[c & 3] = fmaxf(m4[c & 3], v[c]);
             // -inf only for a row that sees no key of this tile (possible with a window)
-            const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+            const float mt = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3])) * sl2;
             if (j == 0) {
                 m_ref = mt;
             } else if (__any_sync(0xffffffffu, mt > m_ref + kRescaleThreshold)) {
@@ -460,7 +505,7 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
                 l *= corr;
                 m_ref = m_new;
 #pragma unroll 1
-                for (int c = 0; c < HD / 16; ++c) {              // 16 columns at a time: S is still live
+                for (int c = 0; c < HD / 16; ++c) {
                     uint32_t o[16];
                     tmem_ld16(tO + 16 * c, o);
                     ptx::tc_wait_ld();
@@ -470,28 +515,36 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
                 }
             }
             const float neg = m_ref == -INFINITY ? 0.f : -m_ref;      // no key seen yet: all p are 0
-            float rs[2] = {0.f, 0.f};
-#pragma unroll
-            for (int c32 = 0; c32 < 2; ++c32) {
+            // one packed FMA per key pair, one SFU exponential per key
+            const uint64_t sc2 = f2pack(sl2, sl2), ng2 = f2pack(neg, neg);
+            uint64_t sum2[2] = {f2pack(0.f, 0.f), f2pack(0.f, 0.f)};
+#pragma unroll 1
+            for (int hh = 0; hh < 2; ++hh) {
+                float v[64];
+                load_half(tS + 64 * hh, v);
+                if (masked) mask_half(v, jt * BN + 64 * hh, lim, row_lo);
                 uint32_t pk[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int c = c32 * 64 + 2 * i;
-                    const float a = ptx::ex2(fmaf(v[c], sl2, neg)), bb = ptx::ex2(fmaf(v[c + 1], sl2, neg));
-                    rs[i & 1] += a + bb;
-                    pk[i] = pack2<T>(a, bb);
-                }
-                tmem_st32(tS + 32 * c32, pk);                   // P column c holds keys 2c, 2c+1
+                for (int i = 0; i < 32; ++i)
+                    pk[i] = exp2_pair<T>(ffma2(f2pack(v[2 * i], v[2 * i + 1]), sc2, ng2), sum2[i & 1]);
+                // P column c holds keys 2c, 2c+1: half hh goes to columns 32 hh .. 32 hh + 31,
+                // which hold scores this thread has already read
+                tmem_st32(tS + 32 * hh, pk);
             }
-            l += rs[0] + rs[1];
+            {
+                float a0, a1, b0, b1;
+                asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(sum2[0]));
+                asm("mov.b64 {%0, %1}, %2;" : "=f"(b0), "=f"(b1) : "l"(sum2[1]));
+                l += (a0 + a1) + (b0 + b1);
+            }
             ptx::tc_wait_st();
             if (x == 0 && ctx < (jt + 1) * BN) {
                 // V rows past the context (tail of the last page, or never loaded) must be
                 // finite zeros: P is 0 there but 0 * NaN would poison O.  Tile A's warps do it
                 // before PV_A(j), which runs before PV_B(j).
                 const int vs = j % VST;
-                ok = wait_bar(bars.v_full(vs), (j / VST) & 1, abort_flag, p.status);
-                if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
+                ok = warp_wait(bars.kv_full((j + 1) % KST), ((j + 1) / KST) & 1, lane, abort_flag, p.status);
+                if (!ok) break;
                 const int first = ctx - jt * BN;                    // first invalid row of the tile
                 uint4* vt = reinterpret_cast<uint4*>(smem + L::kV + vs * L::kTile);
                 const int tid = threadIdx.x - kSoftWarp0 * 32, per = (BN - first) * 8;
@@ -506,12 +559,17 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
             if (lane == 0) ptx::mbar_arrive(bars.p_full(x));       // one arrival per warp
         }
         // epilogue: O / l -> out
-        if (ok) ok = wait_bar(bars.o_full(x), 0, abort_flag, p.status);
-        if (__all_sync(0xffffffffu, ok)) {
+        if (ok) ok = warp_wait(bars.o_full(x), 0, lane, abort_flag, p.status);
+        if (ok) {
+            // The output rows go through shared memory (this tile's Q buffer, free once
+            // its last S MMA is done, which o_full implies) so that the global stores are
+            // whole rows: each thread writes its own row into the staging area (16-byte
+            // chunk c of row r at chunk position c ^ (r % NCH): conflict-free), then the
+            // warp writes its 32 rows out with consecutive lanes on consecutive chunks.
+            constexpr int RB = HD * 2, NCH = RB / 16;               // bytes and 16-byte chunks per row
             ptx::tc_fence_after();
             const float inv = 1.f / l;
-            const bool store = r0 + row < n;
-            T* out = static_cast<T*>(p.out) + (static_cast<size_t>(q0 + r0 + row) * Hq + h0 + x) * HD;
+            uint8_t* stage = smem + L::kQ + x * L::kTile + quarter * 32 * RB;
 #pragma unroll
             for (int c = 0; c < HD / 32; ++c) {
                 uint32_t o[32];
@@ -521,15 +579,24 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
                     wv[i] = pack2<T>(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-                if (store) {
-                    uint4* dst = reinterpret_cast<uint4*>(out + 32 * c);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
+                for (int i = 0; i < 4; ++i) {
+                    const int cc = 4 * c + i;
+                    *reinterpret_cast<uint4*>(stage + lane * RB + ((cc ^ (lane % NCH)) * 16)) =
+                        make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
                 }
             }
+            __syncwarp();
+            T* out = static_cast<T*>(p.out);
+#pragma unroll
+            for (int it = 0; it < NCH; ++it) {
+                const int idx = it * 32 + lane, rr = idx / NCH, c = idx % NCH;
+                const int tr = r0 + quarter * 32 + rr;                  // row within the chunk
+                const uint4 val = *reinterpret_cast<const uint4*>(stage + rr * RB + ((c ^ (rr % NCH)) * 16));
+                if (tr < n)
+                    *reinterpret_cast<uint4*>(out + (static_cast<size_t>(q0 + tr) * Hq + h0 + x) * HD + c * 8) = val;
+            }
         }
-    }
-
     }
 
     ptx::tc_fence_before();
