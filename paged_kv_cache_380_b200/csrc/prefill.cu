@@ -74,7 +74,7 @@ struct Layout {
     static constexpr int kK = kQ + NT * kTile;
     static constexpr int kV = kK + KST * kTile;
     static constexpr int kBar = kV + VST * kTile;
-    static constexpr int kNumBars = 1 + KST + VST + 2 * KST + 2 + VST + 2 + 1;
+    static constexpr int kNumBars = 21;
     static constexpr int kEnd = kBar + kNumBars * 8 + 16;   // + TMEM address, abort flag
     // The CTA holds all of TMEM, so only one may run per SM: ask for more than
     // half of the SM's shared memory even when the tiles need less.
@@ -95,8 +95,12 @@ struct Bars {
     __device__ __forceinline__ uint32_t pv_done(int s) const { return at(3 + 3 * KST + VST + s); }
     __device__ __forceinline__ uint32_t o_full(int x) const { return at(3 + 3 * KST + 2 * VST + x); }
     __device__ __forceinline__ uint32_t mma_done() const { return at(5 + 3 * KST + 2 * VST); }
+    // a unit's epilogue is done (O read, its staging area drained); alternates by unit
+    // parity so that the V producer, which may wait for a unit one behind, is never
+    // two phases late
+    __device__ __forceinline__ uint32_t o_empty(int uc) const { return at(6 + 3 * KST + 2 * VST + (uc & 1)); }
 };
-static_assert(5 + 3 * KST + 2 * VST + 1 == 1 + KST + VST + 2 * KST + 2 + VST + 2 + 1, "barrier count");
+static_assert(6 + 3 * KST + 2 * VST + 2 == 21, "barrier count");
 
 // sm_100 shared-memory matrix descriptor: start, leading and stride byte
 // offsets (>> 4), version 1, SWIZZLE_128B layout.
@@ -158,11 +162,17 @@ __device__ __forceinline__ void load_half(uint32_t taddr, float (&v)[64]) {
 #pragma unroll
     for (int c = 0; c < 64; ++c) v[c] = __uint_as_float(r[c]);
 }
-// Scores of keys outside lo .. lim (key of column c is key0 + c) become -inf.
-__device__ __forceinline__ void mask_half(float (&v)[64], int key0, int lim, int lo) {
+// Scores of keys outside lo .. lim (key of column c is key0 + c) become -inf; without a
+// window only the upper bound can cut (one compare per element).
+__device__ __forceinline__ void mask_half(float (&v)[64], int key0, int lim, int lo, bool window) {
+    const int hi = lim - key0, lw = lo - key0;
+    if (!window) {
 #pragma unroll
-    for (int c = 0; c < 64; ++c)
-        if (key0 + c > lim || key0 + c < lo) v[c] = -INFINITY;
+        for (int c = 0; c < 64; ++c) v[c] = c > hi ? -INFINITY : v[c];
+    } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) v[c] = (c > hi || c < lw) ? -INFINITY : v[c];
+    }
 }
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
@@ -236,6 +246,63 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int lan
     return __all_sync(0xffffffffu, ok);
 }
 
+// One work unit: a 128-row query tile of NT query heads (h0 ..) of sequence b.
+// Units are numbered with the query-tile index varying slowest and reversed, so
+// that lower numbers are the longer (later, more keys) tiles.
+struct Unit {
+    int h0, b, kvh, q0, n, ctx, r0;
+    int t_first, n_tiles;            // 128-key tiles t_first .. t_first + n_tiles - 1
+    int min_lim, lo_mask;            // masking bounds shared by the tile's rows
+    bool valid;
+};
+
+// The three per-sequence values a unit needs, loaded one unit ahead of their use
+// so that each role's walk over its units never waits on them.
+struct UnitLoad {
+    int q0, q1, ctx;
+};
+template <int NT>
+__device__ __forceinline__ UnitLoad unit_load(const PrefillParams& p, int u, int num_units) {
+    if (u >= num_units) return UnitLoad{0, 0, 0};
+    const int b = (u / (p.num_q_heads / NT)) % p.num_seqs;
+    return UnitLoad{__ldg(p.q_start + b), __ldg(p.q_start + b + 1), __ldg(p.context_lens + b)};
+}
+
+template <int NT>
+__device__ __forceinline__ Unit unit_of(const PrefillParams& p, int u, int num_qt, const UnitLoad& ld, bool report) {
+    Unit w{};
+    const int hp_count = p.num_q_heads / NT;
+    const int hp = u % hp_count, rest = u / hp_count;
+    w.b = rest % p.num_seqs;
+    const int qt = num_qt - 1 - rest / p.num_seqs;
+    w.h0 = hp * NT;
+    w.kvh = w.h0 / (p.num_q_heads / p.num_kv_heads);
+    w.q0 = ld.q0;
+    w.n = ld.q1 - ld.q0;
+    w.ctx = ld.ctx;
+    w.r0 = qt * BM;
+    w.valid = false;
+    if (w.r0 >= w.n) return w;
+    if (w.n > w.ctx || w.ctx > p.max_pages_per_seq * p.page_size || w.q0 < 0 || w.q0 + w.n > p.total_q) {
+        if (report) record_error(p.status, PKV_ERR_DEVICE_RANGE, w.ctx);
+        return w;
+    }
+    const int last_row = min(w.r0 + BM, w.n) - 1;
+    const int max_key = p.causal ? w.ctx - w.n + last_row : w.ctx - 1;
+    w.min_lim = p.causal ? w.ctx - w.n + w.r0 : w.ctx - 1;   // every row of the tile sees keys <= this
+    // Local attention (window ww > 0): a row at position pos sees keys pos-ww+1 .. pos
+    // (pos-ww+1 .. ctx-1 without the causal mask), so the tile's key range starts at
+    // the first row's lower bound, and keys below the last row's lower bound need
+    // the lower-edge mask.
+    const int ww = p.window;
+    const int key_lo = ww > 0 ? max(0, w.ctx - w.n + w.r0 - ww + 1) : 0;
+    w.lo_mask = ww > 0 ? max(0, w.ctx - w.n + last_row - ww + 1) : 0;
+    w.t_first = key_lo / BN;
+    w.n_tiles = max_key / BN + 1 - w.t_first;
+    w.valid = true;
+    return w;
+}
+
 // The MMA issuer.  One code path serves every ring slot: a slot only moves the
 // shared-memory start address, i.e. adds a constant to the low word of the
 // descriptor (the address field holds addr >> 4 in 14 bits, and shared memory
@@ -264,7 +331,7 @@ struct Issuer {
         }
         ptx::tc_commit(bars.s_full(x, ks));
     }
-    // O_x (+)= P_x V[stage vs]; the first key tile overwrites O.
+    // O_x (+)= P_x V[stage vs]; the first key tile of a unit overwrites O.
     __device__ __forceinline__ void pv(int x, int vs, bool acc) const {
         constexpr uint32_t id = idesc_f16<T>(BM, HD, 1);
         const uint64_t b = dv + static_cast<uint64_t>((vs * L::kTile) >> 4);
@@ -273,71 +340,55 @@ struct Issuer {
             ptx::tc_mma_ts(kOCol + x * 128, static_cast<uint32_t>(x * 128 + kk * 8), b + static_cast<uint64_t>((kk * 2048) >> 4),
                            id, (acc || kk > 0) ? 1u : 0u);
     }
-    // Key tile j: PV_A(j) S_A(j+1) [PV_B(j) S_B(j+1)].  Three barrier probes per key tile
-    // (P_A, the K/V step, P_B): each probe costs the tensor pipe about as much as three
-    // MMAs, so there are no others.
-    __device__ void run(int n) const {
-        if (!wait(bars.q_full(), 0) || !wait(bars.kv_full(0), 0)) return;
+    // One unit of n key tiles, global tiles g0 .. g0+n-1: S_A(0) [S_B(0)], then per key
+    // tile j: PV_A(j) S_A(j+1) [PV_B(j) S_B(j+1)].  Three barrier probes per key tile (P_A,
+    // the K/V step, P_B): each probe costs the tensor pipe about as much as three MMAs.
+    // uc = units this CTA has issued before (the Q, O-ready and O-read barriers' phase).
+    __device__ bool unit(int g0, int n, int uc) const {
+        if (!wait(bars.q_full(), uc & 1)) return false;
+        if (g0 == 0 && !wait(bars.kv_full(0), 0)) return false;   // later units: waited by the last step
         ptx::tc_fence_after();
-        for (int x = 0; x < NT; ++x) s(x, 0);
-        int vs = 0, ks = 0;                                      // j % VST, j % KST
+        for (int x = 0; x < NT; ++x) s(x, g0 % KST);
         for (int j = 0; j < n; ++j) {
-            const int ks1 = ks + 1 == KST ? 0 : ks + 1;
+            const int g = g0 + j, vs = g % VST, ks1 = (g + 1) % KST;
             const bool more = j + 1 < n;
-            // load step j+1 holds V tile j (for PV) and K tile j+1 (for the next S)
-            if (!wait(bars.p_full(0), j & 1) || !wait(bars.kv_full(ks1), ((j + 1) / KST) & 1)) return;
+            // load step g+1 holds V tile g (for PV) and K tile g+1 (for the next S)
+            if (!wait(bars.p_full(0), g & 1) || !wait(bars.kv_full(ks1), ((g + 1) / KST) & 1)) return false;
+            // the unit's first P.V overwrites O: the previous unit's epilogue must have read it
+            if (j == 0 && uc > 0 && !wait(bars.o_empty(uc - 1), ((uc - 1) >> 1) & 1)) return false;
             ptx::tc_fence_after();
             pv(0, vs, j > 0);
             if (NT == 1) ptx::tc_commit(bars.pv_done(vs));
             if (!more) ptx::tc_commit(bars.o_full(0));
             if (more) s(0, ks1);
             if (NT == 2) {
-                if (!wait(bars.p_full(1), j & 1)) return;
+                if (!wait(bars.p_full(1), g & 1)) return false;
                 ptx::tc_fence_after();
                 pv(1, vs, j > 0);
                 ptx::tc_commit(bars.pv_done(vs));
                 if (!more) ptx::tc_commit(bars.o_full(1));
                 if (more) s(1, ks1);
             }
-            static_assert(VST == 2, "V ring of two stages");
-            vs ^= 1;
-            ks = ks1;
         }
+        return true;
     }
 };
+
+// Persistent: one CTA per SM walks the work units u = blockIdx.x, + gridDim.x, ...
+// (heaviest first).  The rings, the barriers' phases and the key-tile count g run
+// on across units, so the next unit's Q and first K/V tiles load while the current
+// unit finishes, and its first S MMAs overlap the current unit's epilogue.
 template <typename T, int HD, int NT>
 __global__ void __launch_bounds__(kThreads, 1)
-prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
+prefill_tc_kernel(const PrefillParams p, int num_qt, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
     using L = Layout<HD, NT>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = ptx::smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-    const int qt = static_cast<int>(gridDim.z) - 1 - static_cast<int>(blockIdx.z);   // heaviest tiles first
-    const int h0 = blockIdx.x * NT, b = blockIdx.y;
-    const int Hq = p.num_q_heads, kvh = h0 / (Hq / p.num_kv_heads), ps = p.page_size;
-    const int q0 = __ldg(p.q_start + b), n = __ldg(p.q_start + b + 1) - q0;
-    const int ctx = __ldg(p.context_lens + b);
-    const int r0 = qt * BM;
-    if (r0 >= n) return;                                        // whole CTA, before any barrier
-    if (n > ctx || ctx > p.max_pages_per_seq * ps || q0 < 0 || q0 + n > p.total_q) {
-        if (threadIdx.x == 0) record_error(p.status, PKV_ERR_DEVICE_RANGE, ctx);
-        return;
-    }
-    const int last_row = min(r0 + BM, n) - 1;
-    const int max_key = p.causal ? ctx - n + last_row : ctx - 1;
-    const int min_lim = p.causal ? ctx - n + r0 : ctx - 1;      // every row of the tile sees keys <= this
-    // Local attention (window w > 0): a row at position pos sees keys pos-w+1 .. pos
-    // (pos-w+1 .. ctx-1 without the causal mask), so the tile's key range starts at
-    // the first row's lower bound, and keys below the last row's lower bound need
-    // the lower-edge mask.
-    const int w = p.window;
-    const int key_lo = w > 0 ? max(0, ctx - n + r0 - w + 1) : 0;
-    const int lo_mask = w > 0 ? max(0, ctx - n + last_row - w + 1) : 0;
-    const int t_first = key_lo / BN;
-    const int n_tiles = max_key / BN + 1 - t_first;
+    const int num_units = (p.num_q_heads / NT) * p.num_seqs * num_qt;
+    const int Hq = p.num_q_heads, ps = p.page_size;
 
     const Bars bars{sbase + L::kBar};
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBar + L::kNumBars * 8);
@@ -353,6 +404,7 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
         for (int x = 0; x < 2; ++x) {
             ptx::mbar_init(bars.p_full(x), 4);                  // one arrival per softmax warp
             ptx::mbar_init(bars.o_full(x), 1);
+            ptx::mbar_init(bars.o_empty(x), 4 * NT);            // one arrival per softmax warp
         }
         ptx::mbar_init(bars.mma_done(), 1);
         *abort_flag = 0;
@@ -374,75 +426,92 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
 
     if (warp == kKWarp || warp == kVWarp) {
         // ------------------------------ TMA producers ------------------------------
-        // A key tile is 8 page groups of 16 rows x NH column atoms: one box per lane.
-        // K runs up to KST tiles ahead of the S MMAs, V up to VST tiles ahead of PV.
+        // Load step t carries K tile t (K warp) and V tile t-1 (V warp: V runs one tile
+        // behind K) on kv_full(t % KST); t counts key tiles across all units of this
+        // CTA.  A key tile is 8 page groups of 16 rows x NH column atoms: one box per
+        // lane.  The K warp also loads each unit's Q tiles, once the previous unit's
+        // last S MMA has read them.
         const bool is_k = warp == kKWarp;
         const int nst = is_k ? KST : VST;
         const CUtensorMap* map = is_k ? &tm_k : &tm_v;
         const uint32_t ring = sbase + (is_k ? L::kK : L::kV);
-        if (lane == 0) {
-            ptx::prefetch_tmap(map);
-            if (is_k) {
-                ptx::prefetch_tmap(&tm_q);
-                ptx::mbar_arrive_expect_tx(bars.q_full(), NT * L::kTile);
-                for (int x = 0; x < NT; ++x)
-                    for (int a = 0; a < L::NH; ++a)
-                        ptx::tma_load_3d(sbase + L::kQ + x * L::kTile + a * kAtom, &tm_q, bars.q_full(), 64 * a,
-                                         h0 + x, q0 + r0);
-            }
-        }
         const int group = lane / L::NH, half = lane % L::NH;
         const bool my_lane = group < 8;
-        const int32_t* bt = p.block_tables + static_cast<size_t>(b) * p.max_pages_per_seq;
-        // Load step t: the K warp loads K tile t, the V warp V tile t-1 (V runs one tile
-        // behind K), both onto kv_full(t % KST); a warp with no tile at this step just
-        // arrives.  Page indices are read one tile ahead of their use.
-        const int lag = is_k ? 0 : 1;
-        auto page_of = [&](int u) -> int {
-            const int key0 = (t_first + u) * BN + 16 * group;
-            return (my_lane && u >= 0 && u < n_tiles && key0 < ctx) ? __ldg(bt + key0 / ps) : -1;
-        };
-        int pg = page_of(-lag);
-        int t = 0;
-        for (; t <= n_tiles; ++t) {
-            const int u = t - lag;                                  // tile this warp loads at step t
-            const int pg_next = page_of(u + 1);
-            const uint32_t full = bars.kv_full(t % KST);
-            if (u < 0 || u >= n_tiles) {
-                if (lane == 0) ptx::mbar_arrive(full);
-                pg = pg_next;
-                continue;
-            }
-            const int key0 = (t_first + u) * BN + 16 * group;
-            int row = -1;
-            if (my_lane && key0 < ctx) {
-                if (pg < 0 || pg >= p.num_pages) {
-                    if (half == 0) record_error(p.status, PKV_ERR_DEVICE_RANGE, pg);
-                } else {
-                    row = pg * ps + key0 % ps;
+        if (lane == 0) {
+            ptx::prefetch_tmap(map);
+            if (is_k) ptx::prefetch_tmap(&tm_q);
+            else ptx::mbar_arrive(bars.kv_full(0));             // step 0 carries no V tile
+        }
+        int g = 0, uc = 0;
+        int end_g[2] = {-8, -8};            // last key tile of the units with uc parity 0 / 1
+        bool ok = true;
+        UnitLoad ld = unit_load<NT>(p, blockIdx.x, num_units);
+        for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+            const Unit w = unit_of<NT>(p, u, num_qt, ld, is_k && lane == 0);
+            ld = unit_load<NT>(p, u + gridDim.x, num_units);
+            if (!w.valid) continue;
+            if (is_k) {
+                if (uc > 0) {
+                    // Q buffers free: the previous unit's last S MMA (of the last tile) is done
+                    const int gl = g - 1;
+                    ok = warp_wait(bars.s_full(NT - 1, gl % KST), (gl / KST) & 1, lane, abort_flag, p.status);
+                    if (!ok) break;
+                }
+                if (lane == 0) {
+                    ptx::mbar_arrive_expect_tx(bars.q_full(), NT * L::kTile);
+                    for (int x = 0; x < NT; ++x)
+                        for (int a = 0; a < L::NH; ++a)
+                            ptx::tma_load_3d(sbase + L::kQ + x * L::kTile + a * kAtom, &tm_q, bars.q_full(), 64 * a,
+                                             w.h0 + x, w.q0 + w.r0);
                 }
             }
-            const int st = u % nst;
-            bool ok = true;
-            if (u >= nst) {
-                // a K stage is free once S of the last tile KST key tiles back is done,
-                // a V stage once PV of the last tile VST key tiles back is done
-                const int prev = u - nst;
-                ok = warp_wait(is_k ? bars.s_full(NT - 1, st) : bars.pv_done(st), (prev / nst) & 1, lane, abort_flag,
-                               p.status);
+            const int32_t* bt = p.block_tables + static_cast<size_t>(w.b) * p.max_pages_per_seq;
+            for (int j = 0; j < w.n_tiles; ++j, ++g) {
+                const int key0 = (w.t_first + j) * BN + 16 * group;
+                const int pg = (my_lane && key0 < w.ctx) ? __ldg(bt + key0 / ps) : -1;
+                const int st = g % nst;
+                if (g >= nst) {
+                    // a K stage is free once S of the last tile KST key tiles back is done,
+                    // a V stage once PV of the last tile VST key tiles back is done
+                    const int prev = g - nst;
+                    ok = warp_wait(is_k ? bars.s_full(NT - 1, st) : bars.pv_done(st), (prev / nst) & 1, lane,
+                                   abort_flag, p.status);
+                    // a V stage that held a unit's last tile is that unit's epilogue staging
+                    // area until its epilogue is done
+                    for (int e = 0; e < 2 && ok && !is_k; ++e)
+                        if (end_g[e] == prev) {
+                            const int ue = uc - 1 - ((uc - 1 - e) & 1);   // the unit with parity e
+                            ok = warp_wait(bars.o_empty(ue), (ue >> 1) & 1, lane, abort_flag, p.status);
+                        }
+                    if (!ok) break;
+                }
+                int row = -1;
+                if (my_lane && key0 < w.ctx) {
+                    if (pg < 0 || pg >= p.num_pages) {
+                        if (half == 0) record_error(p.status, PKV_ERR_DEVICE_RANGE, pg);
+                    } else {
+                        row = pg * ps + key0 % ps;
+                    }
+                }
+                const unsigned nbox = __popc(__ballot_sync(0xffffffffu, row >= 0));
+                const uint32_t full = bars.kv_full((is_k ? g : g + 1) % KST);
+                if (lane == 0) ptx::mbar_arrive_expect_tx(full, nbox * 16 * 128);
+                __syncwarp();
+                if (row >= 0)
+                    ptx::tma_load_3d(ring + st * L::kTile + half * kAtom + group * 2048, map, full, 64 * half, w.kvh,
+                                     row);
             }
-            if (!ok) break;
-            const unsigned nbox = __popc(__ballot_sync(0xffffffffu, row >= 0));
-            if (lane == 0) ptx::mbar_arrive_expect_tx(full, nbox * 16 * 128);
-            __syncwarp();
-            if (row >= 0)
-                ptx::tma_load_3d(ring + st * L::kTile + half * kAtom + group * 2048, map, full, 64 * half, kvh, row);
-            pg = pg_next;
+            end_g[uc & 1] = g - 1;
+            ++uc;
         }
+        // the step after the last tile carries no K tile
+        if (ok && is_k && lane == 0) ptx::mbar_arrive(bars.kv_full(g % KST));
         if (*abort_flag && lane == 0) {
             // let the copies this warp issued land before the CTA's shared memory is released
-            for (int v = max(0, t - KST); v < t; ++v) ptx::mbar_wait(bars.kv_full(v % KST), (v / KST) & 1, kSpinLimit >> 4);
-            if (is_k) ptx::mbar_wait(bars.q_full(), 0, kSpinLimit >> 4);
+            const int last = is_k ? g : g + 1;
+            for (int v = max(0, last - KST); v < last; ++v)
+                ptx::mbar_wait(bars.kv_full(v % KST), (v / KST) & 1, kSpinLimit >> 4);
+            if (is_k && uc > 0) ptx::mbar_wait(bars.q_full(), (uc - 1) & 1, kSpinLimit >> 4);
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------ MMA issuer ------------------------------
@@ -454,7 +523,16 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
             mma.bars = bars;
             mma.abort_flag = abort_flag;
             mma.status = p.status;
-            mma.run(n_tiles);
+            int g = 0, uc = 0;
+            UnitLoad ld = unit_load<NT>(p, blockIdx.x, num_units);
+            for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+                const Unit w = unit_of<NT>(p, u, num_qt, ld, false);
+                ld = unit_load<NT>(p, u + gridDim.x, num_units);
+                if (!w.valid) continue;
+                if (!mma.unit(g, w.n_tiles, uc)) break;
+                g += w.n_tiles;
+                ++uc;
+            }
             // drain: every tcgen05 op issued by this thread completes before TMEM is freed
             ptx::tc_commit(bars.mma_done());
             ptx::mbar_wait(bars.mma_done(), 0, kSpinLimit);
@@ -466,136 +544,156 @@ prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tm_
         const int row = quarter * 32 + lane;                     // TMEM lane == tile row
         const uint32_t trow = static_cast<uint32_t>(quarter * 32) << 16;
         const uint32_t tS = trow + x * 128, tO = trow + kOCol + x * 128;
-        const int pos = ctx - n + r0 + row;
-        const int lim = p.causal ? min(pos, ctx - 1) : ctx - 1;
-        const int row_lo = w > 0 ? max(0, pos - w + 1) : 0;      // this row's first key
         const float sl2 = p.scale_log2;
-        float m_ref = -INFINITY, l = 0.f;
+        int g = 0, uc = 0;
         bool ok = true;
-        for (int j = 0; j < n_tiles; ++j) {
-            ok = warp_wait(bars.s_full(x, j % KST), (j / KST) & 1, lane, abort_flag, p.status);
+        UnitLoad ld = unit_load<NT>(p, blockIdx.x, num_units);
+        for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+            const Unit w = unit_of<NT>(p, u, num_qt, ld, false);
+            ld = unit_load<NT>(p, u + gridDim.x, num_units);
+            if (!w.valid) continue;
+            const int pos = w.ctx - w.n + w.r0 + row;
+            const int lim = p.causal ? min(pos, w.ctx - 1) : w.ctx - 1;
+            const int row_lo = p.window > 0 ? max(0, pos - p.window + 1) : 0;   // this row's first key
+            float m_ref = -INFINITY, l = 0.f;
+            for (int j = 0; j < w.n_tiles; ++j, ++g) {
+                ok = warp_wait(bars.s_full(x, g % KST), (g / KST) & 1, lane, abort_flag, p.status);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                // Two passes over the row in 64-column halves (one compact loop body each; S
+                // is read from TMEM twice, which costs a few dozen cycles): the row max, then
+                // P = 2^(s * scale - m) written back over the first half of the S columns.
+                const int jt = w.t_first + j;
+                const bool masked = jt * BN + BN - 1 > w.min_lim || jt * BN < w.lo_mask;   // diagonal / last / window edge
+                float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    #pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    float v[64];
+                    load_half(tS + 64 * hh, v);
+                    if (masked) mask_half(v, jt * BN + 64 * hh, lim, row_lo, p.window > 0);
+                    // four independent max chains keep the reduction's latency short
+    #pragma unroll
+                    for (int c = 0; c < 64; c += 8) {
+    #pragma unroll
+                        for (int k = 0; k < 4; ++k) mc[k] = max3(mc[k], v[c + 2 * k], v[c + 2 * k + 1]);
+                    }
+                }
+                // -inf only for a row that sees no key of this tile (possible with a window)
+                const float mt = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3])) * sl2;
+                if (j == 0) {
+                    m_ref = mt;
+                } else if (__any_sync(0xffffffffu, mt > m_ref + kRescaleThreshold)) {
+                    // S_X(j) completed after PV_X(j-1) (same issuer, in order), so O_X is settled
+                    const float m_new = fmaxf(m_ref, mt);
+                    const float corr = m_new == -INFINITY ? 1.f : ptx::ex2(m_ref - m_new);
+                    l *= corr;
+                    m_ref = m_new;
+    #pragma unroll 1
+                    for (int c = 0; c < HD / 16; ++c) {
+                        uint32_t o[16];
+                        tmem_ld16(tO + 16 * c, o);
+                        ptx::tc_wait_ld();
+    #pragma unroll
+                        for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
+                        ptx::tmem_st16(tO + 16 * c, o);
+                    }
+                }
+                const float neg = m_ref == -INFINITY ? 0.f : -m_ref;      // no key seen yet: all p are 0
+                // one packed FMA per key pair, one SFU exponential per key
+                const uint64_t sc2 = f2pack(sl2, sl2), ng2 = f2pack(neg, neg);
+                uint64_t sum2[2] = {f2pack(0.f, 0.f), f2pack(0.f, 0.f)};
+    #pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    float v[64];
+                    load_half(tS + 64 * hh, v);
+                    if (masked) mask_half(v, jt * BN + 64 * hh, lim, row_lo, p.window > 0);
+                    uint32_t pk[32];
+    #pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        pk[i] = exp2_pair<T>(ffma2(f2pack(v[2 * i], v[2 * i + 1]), sc2, ng2), sum2[i & 1]);
+                    // P column c holds keys 2c, 2c+1: half hh goes to columns 32 hh .. 32 hh + 31,
+                    // which hold scores this thread has already read
+                    tmem_st32(tS + 32 * hh, pk);
+                }
+                {
+                    float a0, a1, b0, b1;
+                    asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(sum2[0]));
+                    asm("mov.b64 {%0, %1}, %2;" : "=f"(b0), "=f"(b1) : "l"(sum2[1]));
+                    l += (a0 + a1) + (b0 + b1);
+                }
+                ptx::tc_wait_st();
+                if (x == 0 && w.ctx < (jt + 1) * BN) {
+                    // V rows past the context (tail of the last page, or never loaded) must be
+                    // finite zeros: P is 0 there but 0 * NaN would poison O.  Tile A's warps do it
+                    // before PV_A(j), which runs before PV_B(j).
+                    const int vs = g % VST;
+                    ok = warp_wait(bars.kv_full((g + 1) % KST), ((g + 1) / KST) & 1, lane, abort_flag, p.status);
+                    if (!ok) break;
+                    const int first = w.ctx - jt * BN;                  // first invalid row of the tile
+                    uint4* vt = reinterpret_cast<uint4*>(smem + L::kV + vs * L::kTile);
+                    const int tid = threadIdx.x - kSoftWarp0 * 32, per = (BN - first) * 8;
+                    for (int idx = tid; idx < L::NH * per; idx += 128) {
+                        const int a = idx / per, rem = idx % per;
+                        vt[(a * kAtom + (first + rem / 8) * 128) / 16 + rem % 8] = make_uint4(0, 0, 0, 0);
+                    }
+                    ptx::fence_proxy_async_smem();
+                }
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bars.p_full(x));       // one arrival per warp
+            }
+            if (!ok) break;
+            // epilogue: O / l -> out.  Every P.V of the unit is done once the last tile's
+            // o_full has fired (commits track all earlier MMAs), so the V stage of the
+            // unit's last key tile is free: the rows go through it, a column chunk at a
+            // time (each warp 32 rows x CW columns; 16-byte chunk c of a row at position
+            // c ^ (row % CCH), conflict-free), and leave as whole row segments.
+            ok = warp_wait(bars.o_full(NT - 1), uc & 1, lane, abort_flag, p.status);
             if (!ok) break;
             ptx::tc_fence_after();
-            // Two passes over the row in 64-column halves (one compact loop body each; S
-            // is read from TMEM twice, which costs a few dozen cycles): the row max, then
-            // P = 2^(s * scale - m) written back over the first half of the S columns.
-            const int jt = t_first + j;
-            const bool masked = jt * BN + BN - 1 > min_lim || jt * BN < lo_mask;   // diagonal / last / window edge
-            float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-            for (int hh = 0; hh < 2; ++hh) {
-                float v[64];
-                load_half(tS + 64 * hh, v);
-                if (masked) mask_half(v, jt * BN + 64 * hh, lim, row_lo);
-                // four independent max chains keep the reduction's latency short
-#pragma unroll
-                for (int c = 0; c < 64; c += 8) {
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) mc[k] = max3(mc[k], v[c + 2 * k], v[c + 2 * k + 1]);
-                }
-            }
-            // -inf only for a row that sees no key of this tile (possible with a window)
-            const float mt = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3])) * sl2;
-            if (j == 0) {
-                m_ref = mt;
-            } else if (__any_sync(0xffffffffu, mt > m_ref + kRescaleThreshold)) {
-                // S_X(j) completed after PV_X(j-1) (same issuer, in order), so O_X is settled
-                const float m_new = fmaxf(m_ref, mt);
-                const float corr = m_new == -INFINITY ? 1.f : ptx::ex2(m_ref - m_new);
-                l *= corr;
-                m_ref = m_new;
-#pragma unroll 1
-                for (int c = 0; c < HD / 16; ++c) {
-                    uint32_t o[16];
-                    tmem_ld16(tO + 16 * c, o);
-                    ptx::tc_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
-                    ptx::tmem_st16(tO + 16 * c, o);
-                }
-            }
-            const float neg = m_ref == -INFINITY ? 0.f : -m_ref;      // no key seen yet: all p are 0
-            // one packed FMA per key pair, one SFU exponential per key
-            const uint64_t sc2 = f2pack(sl2, sl2), ng2 = f2pack(neg, neg);
-            uint64_t sum2[2] = {f2pack(0.f, 0.f), f2pack(0.f, 0.f)};
-#pragma unroll 1
-            for (int hh = 0; hh < 2; ++hh) {
-                float v[64];
-                load_half(tS + 64 * hh, v);
-                if (masked) mask_half(v, jt * BN + 64 * hh, lim, row_lo);
-                uint32_t pk[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    pk[i] = exp2_pair<T>(ffma2(f2pack(v[2 * i], v[2 * i + 1]), sc2, ng2), sum2[i & 1]);
-                // P column c holds keys 2c, 2c+1: half hh goes to columns 32 hh .. 32 hh + 31,
-                // which hold scores this thread has already read
-                tmem_st32(tS + 32 * hh, pk);
-            }
             {
-                float a0, a1, b0, b1;
-                asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(sum2[0]));
-                asm("mov.b64 {%0, %1}, %2;" : "=f"(b0), "=f"(b1) : "l"(sum2[1]));
-                l += (a0 + a1) + (b0 + b1);
-            }
-            ptx::tc_wait_st();
-            if (x == 0 && ctx < (jt + 1) * BN) {
-                // V rows past the context (tail of the last page, or never loaded) must be
-                // finite zeros: P is 0 there but 0 * NaN would poison O.  Tile A's warps do it
-                // before PV_A(j), which runs before PV_B(j).
-                const int vs = j % VST;
-                ok = warp_wait(bars.kv_full((j + 1) % KST), ((j + 1) / KST) & 1, lane, abort_flag, p.status);
-                if (!ok) break;
-                const int first = ctx - jt * BN;                    // first invalid row of the tile
-                uint4* vt = reinterpret_cast<uint4*>(smem + L::kV + vs * L::kTile);
-                const int tid = threadIdx.x - kSoftWarp0 * 32, per = (BN - first) * 8;
-                for (int idx = tid; idx < L::NH * per; idx += 128) {
-                    const int a = idx / per, rem = idx % per;
-                    vt[(a * kAtom + (first + rem / 8) * 128) / 16 + rem % 8] = make_uint4(0, 0, 0, 0);
+                constexpr int CW = L::kTile / 512;                   // columns per chunk (64 or 32)
+                constexpr int RB = CW * 2, CCH = RB / 16;             // bytes and 16-byte chunks per row
+                const float inv = 1.f / l;
+                uint8_t* stage = smem + L::kV + ((g - 1) % VST) * L::kTile + (warp - kSoftWarp0) * 32 * RB;
+                T* out = static_cast<T*>(p.out);
+#pragma unroll 1
+                for (int c0 = 0; c0 < HD; c0 += CW) {
+#pragma unroll
+                    for (int c = 0; c < CW / 32; ++c) {
+                        uint32_t o[32];
+                        ptx::tmem_ld32(tO + c0 + 32 * c, o);
+                        ptx::tc_wait_ld();
+                        uint32_t wv[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            wv[i] = pack2<T>(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int cc = 4 * c + i;
+                            *reinterpret_cast<uint4*>(stage + lane * RB + ((cc ^ (lane % CCH)) * 16)) =
+                                make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
+                        }
+                    }
+                    __syncwarp();
+#pragma unroll
+                    for (int it = 0; it < CCH; ++it) {
+                        const int idx = it * 32 + lane, rr = idx / CCH, cc = idx % CCH;
+                        const int tr = w.r0 + quarter * 32 + rr;          // row within the chunk
+                        const uint4 val = *reinterpret_cast<const uint4*>(stage + rr * RB + ((cc ^ (rr % CCH)) * 16));
+                        if (tr < w.n)
+                            *reinterpret_cast<uint4*>(out + (static_cast<size_t>(w.q0 + tr) * Hq + w.h0 + x) * HD + c0 +
+                                                      cc * 8) = val;
+                    }
+                    __syncwarp();
                 }
-                ptx::fence_proxy_async_smem();
             }
+            // O is read and the staging area drained: the next unit's first P.V may overwrite
+            // O, and the V producer may refill the stage
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(bars.p_full(x));       // one arrival per warp
-        }
-        // epilogue: O / l -> out
-        if (ok) ok = warp_wait(bars.o_full(x), 0, lane, abort_flag, p.status);
-        if (ok) {
-            // The output rows go through shared memory (this tile's Q buffer, free once
-            // its last S MMA is done, which o_full implies) so that the global stores are
-            // whole rows: each thread writes its own row into the staging area (16-byte
-            // chunk c of row r at chunk position c ^ (r % NCH): conflict-free), then the
-            // warp writes its 32 rows out with consecutive lanes on consecutive chunks.
-            constexpr int RB = HD * 2, NCH = RB / 16;               // bytes and 16-byte chunks per row
-            ptx::tc_fence_after();
-            const float inv = 1.f / l;
-            uint8_t* stage = smem + L::kQ + x * L::kTile + quarter * 32 * RB;
-#pragma unroll
-            for (int c = 0; c < HD / 32; ++c) {
-                uint32_t o[32];
-                ptx::tmem_ld32(tO + 32 * c, o);
-                ptx::tc_wait_ld();
-                uint32_t wv[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    wv[i] = pack2<T>(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int cc = 4 * c + i;
-                    *reinterpret_cast<uint4*>(stage + lane * RB + ((cc ^ (lane % NCH)) * 16)) =
-                        make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
-                }
-            }
-            __syncwarp();
-            T* out = static_cast<T*>(p.out);
-#pragma unroll
-            for (int it = 0; it < NCH; ++it) {
-                const int idx = it * 32 + lane, rr = idx / NCH, c = idx % NCH;
-                const int tr = r0 + quarter * 32 + rr;                  // row within the chunk
-                const uint4 val = *reinterpret_cast<const uint4*>(stage + rr * RB + ((c ^ (rr % NCH)) * 16));
-                if (tr < n)
-                    *reinterpret_cast<uint4*>(out + (static_cast<size_t>(q0 + tr) * Hq + h0 + x) * HD + c * 8) = val;
-            }
+            if (lane == 0) ptx::mbar_arrive(bars.o_empty(uc));
+            ++uc;
         }
     }
 
@@ -651,10 +749,16 @@ cudaError_t run(const PrefillParams& p, cudaStream_t stream) {
         !make_map(&tk, p.k_pages, dt, HD, p.num_kv_heads, pool_rows, 16) ||
         !make_map(&tv, p.v_pages, dt, HD, p.num_kv_heads, pool_rows, 16))
         return cudaErrorInvalidValue;
-    dim3 grid(p.num_q_heads / NT, p.num_seqs, ceil_div(p.max_q_len, BM));
+    // one persistent CTA per SM (at most one per work unit)
+    const int num_qt = ceil_div(p.max_q_len, BM);
+    const long long units = static_cast<long long>(p.num_q_heads / NT) * p.num_seqs * num_qt;
+    if (units > 0x7fffffffLL) return cudaErrorInvalidValue;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = static_cast<int>(units < sms ? units : sms);
     cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(prefill_tc_kernel<T, HD, NT>), L::kSmem);
     if (e != cudaSuccess) return e;
-    prefill_tc_kernel<T, HD, NT><<<grid, kThreads, L::kSmem, stream>>>(p, tq, tk, tv);
+    prefill_tc_kernel<T, HD, NT><<<grid, kThreads, L::kSmem, stream>>>(p, num_qt, tq, tk, tv);
     return cudaGetLastError();
 }
 
