@@ -49,15 +49,26 @@ constexpr int kChunk = 16;            // tokens per pipeline stage of one warp
 constexpr unsigned kFull = 0xffffffffu;
 
 // int8 code pair (bytes a, b of w, each offset by 128 through w ^ 0x80808080)
-// -> fp16x2, exact: the offset byte u becomes the low mantissa byte of the fp16
-// number 1024 + u (exponent pattern 0x64), then 1152 = 1024 + 128 is subtracted
-// from both halves at once; |code| <= 128 is exact in fp16.
+// -> fp16x2 holding 1152 + code, exact, in one byte permute: the offset byte
+// u = code + 128 becomes the low mantissa byte of the fp16 number 1024 + u
+// (exponent pattern 0x64).
+__device__ __forceinline__ uint32_t s8pair_biased(uint32_t w_biased, uint32_t sel_a, uint32_t sel_b) {
+    return __byte_perm(w_biased, 0x64646464u, sel_a | 0x40u | (sel_b << 8) | 0x4000u);
+}
+// ... and the code itself: 1152 subtracted from both halves (exact in fp16).  Keys
+// use this form: a key bias would add 1152 sum(q) to every score, and removing it
+// after the fp32 accumulation costs precision when |q| is large.
 __device__ __forceinline__ uint32_t s8pair(uint32_t w_biased, uint32_t sel_a, uint32_t sel_b) {
-    const uint32_t h = __byte_perm(w_biased, 0x64646464u, sel_a | 0x40u | (sel_b << 8) | 0x4000u);
+    const uint32_t h = s8pair_biased(w_biased, sel_a, sel_b);
     __half2 x = *reinterpret_cast<const __half2*>(&h);
     x = __hsub2(x, __half2half2(__ushort_as_half(0x6480)));   // 0x6480 = 1152.0
     return *reinterpret_cast<uint32_t*>(&x);
 }
+// Values stay biased: sum_t p_t (v_t + 1152) = sum_t p_t v_t + 1152 sum_t p_t, and
+// sum_t p_t comes from one more MMA per chunk against a matrix of ones (the same fp16
+// P operand, p <= 1), accumulated and rescaled with O and subtracted at the end.
+constexpr float kCodeBias = 1152.f;
+constexpr uint32_t kOnePair = 0x3C003C00u;    // fp16x2 (1, 1)
 
 template <typename QT>
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -219,10 +230,12 @@ decode_mma_kernel(const DecodeParams p) {
     };
 
     float m[NT][2], l[NT][2], o[NT][Cfg::kDT][4];
+    float osum[NT][4];   // INT8: sum over tokens of the fp16 P operand, per head (bias of O)
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
         m[nt][0] = m[nt][1] = -INFINITY;
         l[nt][0] = l[nt][1] = 0.f;
+        osum[nt][0] = osum[nt][1] = osum[nt][2] = osum[nt][3] = 0.f;
 #pragma unroll
         for (int dt = 0; dt < Cfg::kDT; ++dt) o[nt][dt][0] = o[nt][dt][1] = o[nt][dt][2] = o[nt][dt][3] = 0.f;
     }
@@ -316,6 +329,10 @@ decode_mma_kernel(const DecodeParams p) {
                         o[nt][dt][h] *= corr;
                         o[nt][dt][2 + h] *= corr;
                     }
+                    if constexpr (Cfg::kInt8) {
+                        osum[nt][h] *= corr;
+                        osum[nt][2 + h] *= corr;
+                    }
                 }
                 pr[h] = ptx::ex2(x[h] - m[nt][h]);
                 pr[2 + h] = ptx::ex2(x[2 + h] - m[nt][h]);
@@ -347,16 +364,28 @@ decode_mma_kernel(const DecodeParams p) {
                 w0 ^= 0x80808080u; w1 ^= 0x80808080u; w2 ^= 0x80808080u; w3 ^= 0x80808080u;
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    mma16816<MT>(o[nt][U], s8pair(w0, 0, 2), s8pair(w0, 1, 3), s8pair(w1, 0, 2),
-                                 s8pair(w1, 1, 3), pb[nt][0], pb[nt][1]);
-                    mma16816<MT>(o[nt][U + 1], s8pair(w2, 0, 2), s8pair(w2, 1, 3), s8pair(w3, 0, 2),
-                                 s8pair(w3, 1, 3), pb[nt][0], pb[nt][1]);
+                    mma16816<MT>(o[nt][U], s8pair_biased(w0, 0, 2), s8pair_biased(w0, 1, 3), s8pair_biased(w1, 0, 2),
+                                 s8pair_biased(w1, 1, 3), pb[nt][0], pb[nt][1]);
+                    mma16816<MT>(o[nt][U + 1], s8pair_biased(w2, 0, 2), s8pair_biased(w2, 1, 3),
+                                 s8pair_biased(w3, 0, 2), s8pair_biased(w3, 1, 3), pb[nt][0], pb[nt][1]);
                 }
             }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                mma16816<MT>(osum[nt], kOnePair, kOnePair, kOnePair, kOnePair, pb[nt][0], pb[nt][1]);
         }
         __syncwarp();
     }
     ptx::cp_async_wait<0>();
+    if constexpr (Cfg::kInt8) {
+        // O accumulated (v + 1152) p: subtract 1152 sum_t p_t (rows of osum are all equal)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int dt = 0; dt < Cfg::kDT; ++dt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) o[nt][dt][i] -= kCodeBias * osum[nt][i & 1];
+    }
 
     // ---- merge the warps' partial softmax states ----
 #pragma unroll
@@ -542,14 +571,17 @@ __global__ void __launch_bounds__(128) decode_f32_kernel(const DecodeParams p) {
 #ifndef PKV_DECODE_WARPS
 #define PKV_DECODE_WARPS 4
 #endif
-#ifndef PKV_DECODE_STAGES
-#define PKV_DECODE_STAGES 3
-#endif
 constexpr int kWarps = PKV_DECODE_WARPS;    // warps per CTA, each with its own cp.async ring
-constexpr int kStages = PKV_DECODE_STAGES;  // ring depth (16-token chunks)
+// Ring depth (16-token chunks), measured per KV type: with 16-bit pages two stages
+// (64 KB of ring per CTA) let three CTAs share an SM, which beats the deeper ring of
+// two resident CTAs by 2-6% on the decode workloads; int8 pages (4 KB per stage, and
+// register-limited to four CTAs per SM) run best with three.
+template <typename KVT>
+constexpr int stages_for() { return std::is_same<KVT, int8_t>::value ? 3 : 2; }
 
 template <typename QT, typename KVT, int HD, int NT>
 cudaError_t run_mma(const DecodeParams& p, cudaStream_t stream) {
+    constexpr int kStages = stages_for<KVT>();
     using Cfg = DecodeCfg<QT, KVT, HD, NT, kWarps, kStages>;
     auto kern = decode_mma_kernel<QT, KVT, HD, NT, kWarps, kStages>;
     cudaError_t e0 = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), Cfg::kSmem);

@@ -131,3 +131,20 @@ def test_head_dim_64_fp16_large_pages():
 def test_odd_group_sizes(Hq, Hkv):
     # groups of 3 query heads: one query tile per CTA instead of a pair
     run_prefill(case(33 + Hq, chunks=(17, 130, 256), Hq=Hq, Hkv=Hkv, private_prefix=9))
+
+
+# ---- many work units per CTA (the kernel walks its units persistently) --------------
+
+@pytest.mark.parametrize("window", [0, 200])
+def test_many_units_per_cta(window):
+    # 160 sequences with seeded chunk lengths 0..400 and private prefixes: several hundred
+    # (head pair, sequence, query tile) units, many of them empty, walked by each CTA in turn
+    rng = np.random.default_rng(11)
+    chunks = tuple(int(c) for c in rng.integers(0, 400, 160))
+    run_prefill(case(40, chunks=chunks, private_prefix=5, shared_prefix=32, Hq=4, Hkv=2), window=window)
+
+
+def test_many_units_head_dim_64_non_causal():
+    rng = np.random.default_rng(12)
+    chunks = tuple(int(c) for c in rng.integers(1, 300, 120))
+    run_prefill(case(41, chunks=chunks, private_prefix=0, shared_prefix=64, Hq=6, Hkv=3, D=64), causal=False)
