@@ -187,44 +187,65 @@ decode_mma_kernel(const DecodeParams p) {
     }
 
     // ---- per-warp cp.async ring ----
+    // Everything per lane that does not change from chunk to chunk is computed once:
+    // the shared-memory destination of each of the lane's 16-byte copies, their byte
+    // offsets from the chunk's first pool row, and the chunk-relative token row.  Per
+    // chunk only the pool row (read with the page indices, 32 chunks at a time) and
+    // the context test change.
     uint8_t* ring = smem + warp * STAGES * Cfg::kStage;
     const uint32_t ring_s = ptx::smem_u32(ring);
     const uint8_t* kpool = static_cast<const uint8_t*>(p.k_pages);
     const uint8_t* vpool = static_cast<const uint8_t*>(p.v_pages);
     const int32_t* bt = p.block_tables + static_cast<size_t>(b) * p.max_pages_per_seq;
-    int page_reg = 0;
+    constexpr int NI = kChunk * Cfg::kUnits / 32;          // 16-byte copies per lane per tensor
+    uint32_t cp_dst[NI];
+    int32_t cp_off[NI], cp_row[NI];
+#pragma unroll
+    for (int k = 0; k < NI; ++k) {
+        const int x = lane + 32 * k, r = x / Cfg::kUnits, u = x % Cfg::kUnits;
+        cp_row[k] = r;
+        cp_dst[k] = r * Cfg::kRowBytes + ((u ^ (r & 7)) << 4);
+        cp_off[k] = r * Hkv * Cfg::kRowBytes + u * 16;
+    }
+    const int sc_row = lane & 15;                           // INT8 scale copies: token row of this lane
+    int64_t first_row_reg = 0;                              // pool row of chunk (i & ~31) + lane, or -1
+    int issue_slot = 0;
 
     auto issue = [&](int i) {
         if (i < n_mine) {
-            if ((i & 31) == 0) {        // page indices of my next 32 chunks, one per lane
+            if ((i & 31) == 0) {        // first pool rows of my next 32 chunks, one per lane
                 const int j = i + lane;
-                page_reg = j < n_mine ? __ldg(bt + ((c_begin + warp + j * WARPS) * kChunk) / ps) : 0;
+                int64_t fr = 0;
+                if (j < n_mine) {
+                    const int tok = (c_begin + warp + j * WARPS) * kChunk;
+                    const int page = __ldg(bt + tok / ps);
+                    fr = (page >= 0 && page < p.num_pages) ? static_cast<int64_t>(page) * ps + tok % ps : -1;
+                    if (fr < 0) record_error(p.status, PKV_ERR_DEVICE_RANGE, page);
+                }
+                first_row_reg = fr;
             }
-            const int page = __shfl_sync(kFull, page_reg, i & 31);
-            const int tok0 = (c_begin + warp + i * WARPS) * kChunk;
-            const bool page_ok = page >= 0 && page < p.num_pages;
-            if (!page_ok && lane == 0) record_error(p.status, PKV_ERR_DEVICE_RANGE, page);
-            const int64_t row0 = (static_cast<int64_t>(page) * ps + (tok0 % ps)) * Hkv + kvh;
-            const uint32_t sK = ring_s + (i % STAGES) * Cfg::kStage;
+            const int64_t frow = __shfl_sync(kFull, first_row_reg, i & 31);
+            const int rem = frow < 0 ? 0 : ctx - (c_begin + warp + i * WARPS) * kChunk;   // valid rows
+            const int64_t row0 = (frow < 0 ? 0 : frow) * Hkv + kvh;
+            const uint8_t* kb = kpool + row0 * Cfg::kRowBytes;
+            const uint8_t* vb = vpool + row0 * Cfg::kRowBytes;
+            const uint32_t sK = ring_s + issue_slot * Cfg::kStage;
             const uint32_t sV = sK + Cfg::kTile;
 #pragma unroll
-            for (int x = lane; x < kChunk * Cfg::kUnits; x += 32) {
-                const int r = x / Cfg::kUnits, u = x % Cfg::kUnits;
-                const bool ok = page_ok && (tok0 + r < ctx);
-                const int64_t off = (row0 + static_cast<int64_t>(r) * Hkv) * Cfg::kRowBytes + u * 16;
-                const uint32_t dst = r * Cfg::kRowBytes + ((u ^ (r & 7)) << 4);
-                ptx::cp_async16(sK + dst, ok ? kpool + off : kpool, ok ? 16u : 0u);
-                ptx::cp_async16(sV + dst, ok ? vpool + off : vpool, ok ? 16u : 0u);
+            for (int k = 0; k < NI; ++k) {
+                const bool ok = cp_row[k] < rem;
+                ptx::cp_async16(sK + cp_dst[k], ok ? kb + cp_off[k] : kpool, ok ? 16u : 0u);
+                ptx::cp_async16(sV + cp_dst[k], ok ? vb + cp_off[k] : vpool, ok ? 16u : 0u);
             }
             if constexpr (Cfg::kInt8) {   // lanes 0-15: key scales, 16-31: value scales
-                const int r = lane & 15;
-                const bool ok = page_ok && (tok0 + r < ctx);
+                const bool ok = sc_row < rem;
                 const __half* sc = lane < 16 ? p.k_scales : p.v_scales;
-                const uintptr_t a = reinterpret_cast<uintptr_t>(sc + (row0 + static_cast<int64_t>(r) * Hkv));
+                const uintptr_t a = reinterpret_cast<uintptr_t>(sc + (row0 + static_cast<int64_t>(sc_row) * Hkv));
                 ptx::cp_async4(sV + Cfg::kTile + lane * 4,
                                ok ? reinterpret_cast<const void*>(a & ~uintptr_t(3)) : static_cast<const void*>(sc),
                                ok ? 4u : 0u);
             }
+            issue_slot = issue_slot + 1 == STAGES ? 0 : issue_slot + 1;
         }
         ptx::cp_async_commit();
     };
@@ -243,11 +264,12 @@ decode_mma_kernel(const DecodeParams p) {
 #pragma unroll
     for (int i = 0; i < STAGES - 1; ++i) issue(i);
 
+    int use_slot = 0;
     for (int i = 0; i < n_mine; ++i) {
         issue(i + STAGES - 1);
         ptx::cp_async_wait<STAGES - 1>();
         __syncwarp();
-        const uint32_t sK = ring_s + (i % STAGES) * Cfg::kStage;
+        const uint32_t sK = ring_s + use_slot * Cfg::kStage;
         const uint32_t sV = sK + Cfg::kTile;
         const int tok0 = (c_begin + warp + i * WARPS) * kChunk;
 
@@ -292,7 +314,7 @@ decode_mma_kernel(const DecodeParams p) {
             // half is the parity of the element index (slot * Hkv + kvh).  With
             // page_size a multiple of 16 that parity is kvh's for even Hkv and
             // (row + kvh)'s for odd Hkv.
-            const uint8_t* sS = ring + (i % STAGES) * Cfg::kStage + 2 * Cfg::kTile;
+            const uint8_t* sS = ring + use_slot * Cfg::kStage + 2 * Cfg::kTile;
             auto scale_at = [&](int base, int row) {
                 const uint32_t w = *reinterpret_cast<const uint32_t*>(sS + base + row * 4);
                 const int odd = ((Hkv & 1) ? (row + kvh) : kvh) & 1;
@@ -375,6 +397,7 @@ decode_mma_kernel(const DecodeParams p) {
                 mma16816<MT>(osum[nt], kOnePair, kOnePair, kOnePair, kOnePair, pb[nt][0], pb[nt][1]);
         }
         __syncwarp();
+        use_slot = use_slot + 1 == STAGES ? 0 : use_slot + 1;
     }
     ptx::cp_async_wait<0>();
     if constexpr (Cfg::kInt8) {
