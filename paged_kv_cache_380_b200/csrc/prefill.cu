@@ -341,8 +341,9 @@ struct Issuer {
                            id, (acc || kk > 0) ? 1u : 0u);
     }
     // One unit of n key tiles, global tiles g0 .. g0+n-1: S_A(0) [S_B(0)], then per key
-    // tile j: PV_A(j) S_A(j+1) [PV_B(j) S_B(j+1)].  Three barrier probes per key tile (P_A,
-    // the K/V step, P_B): each probe costs the tensor pipe about as much as three MMAs.
+    // tile j: PV_A(j) S_A(j+1) [PV_B(j) S_B(j+1)].  Three barrier probes per key tile (the
+    // K/V step, P_A, P_B): each probe costs the tensor pipe about as much as two MMAs when
+    // nothing is queued behind it.
     // uc = units this CTA has issued before (the Q, O-ready and O-read barriers' phase).
     __device__ bool unit(int g0, int n, int uc) const {
         if (!wait(bars.q_full(), uc & 1)) return false;
@@ -352,10 +353,13 @@ struct Issuer {
         for (int j = 0; j < n; ++j) {
             const int g = g0 + j, vs = g % VST, ks1 = (g + 1) % KST;
             const bool more = j + 1 < n;
-            // load step g+1 holds V tile g (for PV) and K tile g+1 (for the next S)
-            if (!wait(bars.p_full(0), g & 1) || !wait(bars.kv_full(ks1), ((g + 1) / KST) & 1)) return false;
+            // load step g+1 holds V tile g (for PV) and K tile g+1 (for the next S).  It is
+            // probed first: it has normally landed long before, and the tensor pipe idles from
+            // P_A ready until the first P.V is issued, so nothing but that wait sits there.
+            if (!wait(bars.kv_full(ks1), ((g + 1) / KST) & 1)) return false;
             // the unit's first P.V overwrites O: the previous unit's epilogue must have read it
             if (j == 0 && uc > 0 && !wait(bars.o_empty(uc - 1), ((uc - 1) >> 1) & 1)) return false;
+            if (!wait(bars.p_full(0), g & 1)) return false;
             ptx::tc_fence_after();
             pv(0, vs, j > 0);
             if (NT == 1) ptx::tc_commit(bars.pv_done(vs));

@@ -148,3 +148,55 @@ def test_many_units_head_dim_64_non_causal():
     rng = np.random.default_rng(12)
     chunks = tuple(int(c) for c in rng.integers(1, 300, 120))
     run_prefill(case(41, chunks=chunks, private_prefix=0, shared_prefix=64, Hq=6, Hkv=3, D=64), causal=False)
+
+
+# ---- scores whose row maximum keeps rising (the reference-max raise path) ----------
+
+def _to_bits(x: np.ndarray, dtype: str) -> np.ndarray:
+    return W.to_bf16_bits(x) if dtype == "bf16" else x.astype(np.float16).view(np.uint16)
+
+
+def _from_bits(b: np.ndarray, dtype: str) -> np.ndarray:
+    return W.bf16_bits_to_f32(b) if dtype == "bf16" else b.view(np.float16).astype(np.float32)
+
+
+def rising_scores(c, step_log2: float = 12.0):
+    """Rewrite a prefill case so that, for even query heads, the scaled score of key
+    position t grows by about step_log2 (log2 units) every 64 keys: every half of every
+    128-key tile raises the row maximum past the lazy-rescale threshold.  Odd heads see
+    the mirror image (falling scores: the first keys hold the maximum)."""
+    dt, D, ps = c.dtype, c.head_dim, c.page_size
+    rng = np.random.default_rng(5)
+    u = np.ones(D, dtype=np.float32) / np.sqrt(D)
+    slope = step_log2 / 64.0 / (c.scale * np.log2(np.e))         # q.k growth per key
+    q = 0.1 * rng.standard_normal(c.q.shape).astype(np.float32)
+    q[:, 0::2, :] += u
+    q[:, 1::2, :] -= u
+    c.q = _to_bits(q, dt)
+    kp, kn = _from_bits(c.k_pages, dt), _from_bits(c.k_new, dt)
+    for b in range(len(c.context_lens)):
+        ctx, n = int(c.context_lens[b]), int(c.q_start[b + 1] - c.q_start[b])
+        for t in range(ctx):
+            row = slope * t * u + 0.1 * rng.standard_normal((c.num_kv_heads, D)).astype(np.float32)
+            if t < ctx - n:
+                pg = int(c.block_tables[b, t // ps])
+                kp[pg, t % ps] = row
+            else:
+                kn[int(c.q_start[b]) + t - (ctx - n)] = row
+    c.k_pages, c.k_new = _to_bits(kp, dt), _to_bits(kn, dt)
+    return c
+
+
+@pytest.mark.parametrize("dtype,D", [("bf16", 128), ("f16", 128), ("bf16", 64)])
+def test_rising_row_maximum(dtype, D):
+    # chunks over several key tiles, ragged, after shared and private prefixes
+    c = rising_scores(case(50 + D // 64 + (dtype == "f16"), chunks=(300, 129, 40), private_prefix=9,
+                           shared_prefix=64, dtype=dtype, D=D))
+    run_prefill(c)
+
+
+def test_rising_row_maximum_window_and_non_causal():
+    c = rising_scores(case(55, chunks=(260, 77), private_prefix=5, shared_prefix=128))
+    run_prefill(c, window=150)
+    c = rising_scores(case(56, chunks=(260, 77), private_prefix=5, shared_prefix=128))
+    run_prefill(c, causal=False)
