@@ -74,8 +74,9 @@ struct Layout {
     static constexpr int kK = kQ + NT * kTile;
     static constexpr int kV = kK + KST * kTile;
     static constexpr int kBar = kV + VST * kTile;
-    static constexpr int kNumBars = 21;
-    static constexpr int kEnd = kBar + kNumBars * 8 + 16;   // + TMEM address, abort flag
+    static constexpr int kNumBars = 23;
+    static constexpr int kPend = kBar + kNumBars * 8 + 16;  // after the TMEM address and abort flag
+    static constexpr int kEnd = kPend + 8 * 32;             // a pending epilogue's unit, per softmax warp
     // The CTA holds all of TMEM, so only one may run per SM: ask for more than
     // half of the SM's shared memory even when the tiles need less.
     static constexpr int kSmem = kEnd + 1024 > 120 * 1024 ? kEnd + 1024 : 120 * 1024;
@@ -95,12 +96,13 @@ struct Bars {
     __device__ __forceinline__ uint32_t pv_done(int s) const { return at(3 + 3 * KST + VST + s); }
     __device__ __forceinline__ uint32_t o_full(int x) const { return at(3 + 3 * KST + 2 * VST + x); }
     __device__ __forceinline__ uint32_t mma_done() const { return at(5 + 3 * KST + 2 * VST); }
-    // a unit's epilogue is done (O read, its staging area drained); alternates by unit
-    // parity so that the V producer, which may wait for a unit one behind, is never
-    // two phases late
-    __device__ __forceinline__ uint32_t o_empty(int uc) const { return at(6 + 3 * KST + 2 * VST + (uc & 1)); }
+    // a unit's O has been read by its epilogue (the next unit's first P.V may overwrite it),
+    // and the unit's epilogue staging area is drained (the V producer may refill it); both
+    // alternate by unit parity so that a waiter one unit behind is never two phases late
+    __device__ __forceinline__ uint32_t o_read(int uc) const { return at(6 + 3 * KST + 2 * VST + (uc & 1)); }
+    __device__ __forceinline__ uint32_t stage_free(int uc) const { return at(8 + 3 * KST + 2 * VST + (uc & 1)); }
 };
-static_assert(6 + 3 * KST + 2 * VST + 2 == 21, "barrier count");
+static_assert(8 + 3 * KST + 2 * VST + 2 == 23, "barrier count");
 
 // sm_100 shared-memory matrix descriptor: start, leading and stride byte
 // offsets (>> 4), version 1, SWIZZLE_128B layout.
@@ -261,11 +263,18 @@ struct Unit {
 struct UnitLoad {
     int q0, q1, ctx;
 };
+// A read-only global load kept where it is written (volatile): issued a unit ahead, its
+// latency is hidden behind the current unit instead of being moved next to its use.
+__device__ __forceinline__ int ld_early(const int* ptr) {
+    int v;
+    asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(v) : "l"(ptr));
+    return v;
+}
 template <int NT>
 __device__ __forceinline__ UnitLoad unit_load(const PrefillParams& p, int u, int num_units) {
     if (u >= num_units) return UnitLoad{0, 0, 0};
     const int b = (u / (p.num_q_heads / NT)) % p.num_seqs;
-    return UnitLoad{__ldg(p.q_start + b), __ldg(p.q_start + b + 1), __ldg(p.context_lens + b)};
+    return UnitLoad{ld_early(p.q_start + b), ld_early(p.q_start + b + 1), ld_early(p.context_lens + b)};
 }
 
 template <int NT>
@@ -358,7 +367,7 @@ struct Issuer {
             // P_A ready until the first P.V is issued, so nothing but that wait sits there.
             if (!wait(bars.kv_full(ks1), ((g + 1) / KST) & 1)) return false;
             // the unit's first P.V overwrites O: the previous unit's epilogue must have read it
-            if (j == 0 && uc > 0 && !wait(bars.o_empty(uc - 1), ((uc - 1) >> 1) & 1)) return false;
+            if (j == 0 && uc > 0 && !wait(bars.o_read(uc - 1), ((uc - 1) >> 1) & 1)) return false;
             if (!wait(bars.p_full(0), g & 1)) return false;
             ptx::tc_fence_after();
             pv(0, vs, j > 0);
@@ -408,7 +417,8 @@ prefill_tc_kernel(const PrefillParams p, int num_qt, const __grid_constant__ CUt
         for (int x = 0; x < 2; ++x) {
             ptx::mbar_init(bars.p_full(x), 4);                  // one arrival per softmax warp
             ptx::mbar_init(bars.o_full(x), 1);
-            ptx::mbar_init(bars.o_empty(x), 4 * NT);            // one arrival per softmax warp
+            ptx::mbar_init(bars.o_read(x), 4 * NT);             // one arrival per softmax warp
+            ptx::mbar_init(bars.stage_free(x), 4 * NT);
         }
         ptx::mbar_init(bars.mma_done(), 1);
         *abort_flag = 0;
@@ -481,11 +491,11 @@ prefill_tc_kernel(const PrefillParams p, int num_qt, const __grid_constant__ CUt
                     ok = warp_wait(is_k ? bars.s_full(NT - 1, st) : bars.pv_done(st), (prev / nst) & 1, lane,
                                    abort_flag, p.status);
                     // a V stage that held a unit's last tile is that unit's epilogue staging
-                    // area until its epilogue is done
+                    // area until its epilogue has drained it
                     for (int e = 0; e < 2 && ok && !is_k; ++e)
                         if (end_g[e] == prev) {
                             const int ue = uc - 1 - ((uc - 1 - e) & 1);   // the unit with parity e
-                            ok = warp_wait(bars.o_empty(ue), (ue >> 1) & 1, lane, abort_flag, p.status);
+                            ok = warp_wait(bars.stage_free(ue), (ue >> 1) & 1, lane, abort_flag, p.status);
                         }
                     if (!ok) break;
                 }
@@ -551,6 +561,71 @@ prefill_tc_kernel(const PrefillParams p, int num_qt, const __grid_constant__ CUt
         const float sl2 = p.scale_log2;
         int g = 0, uc = 0;
         bool ok = true;
+        // A unit's epilogue runs once the next unit's first key tile is through softmax (or
+        // after the last unit), so that it overlaps the next unit's first MMAs instead of
+        // delaying them: it waits for the unit's last P.V (o_full), reads O into registers,
+        // lets the issuer overwrite O (o_read), then writes O / l out through the V stage of
+        // the unit's last key tile and releases that stage to the V producer (stage_free).
+        // Every P.V of the unit is done once o_full of its last tile has fired (commits track
+        // all earlier MMAs), so that V stage is no longer read.
+        // The pending unit's parameters wait in shared memory (warp-uniform; kept out of the
+        // registers the softmax needs), its row sum in l_pend.
+        struct Pending {
+            int q0, n, r0, h0, g_last, uc;
+        };
+        Pending* pend_s = reinterpret_cast<Pending*>(smem + L::kPend) + (warp - kSoftWarp0);
+        float l_pend = 0.f;
+        bool pending = false;
+        auto epilogue = [&]() -> bool {
+            __syncwarp();
+            const Pending e = *pend_s;
+            if (!warp_wait(bars.o_full(NT - 1), e.uc & 1, lane, abort_flag, p.status)) return false;
+            ptx::tc_fence_after();
+            // O / l is read into registers (packed to T), then the issuer may overwrite O
+            // (o_read) while the rows leave a column chunk at a time (each warp 32 rows x CW
+            // columns; 16-byte chunk c of a row at position c ^ (row % CCH), conflict-free) as
+            // whole row segments.
+            uint32_t ob[HD / 2];
+            const float inv = 1.f / l_pend;
+#pragma unroll
+            for (int c = 0; c < HD / 32; ++c) {
+                uint32_t o[32];
+                ptx::tmem_ld32(tO + 32 * c, o);
+                ptx::tc_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    ob[16 * c + i] = pack2<T>(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bars.o_read(e.uc));
+            constexpr int CW = L::kTile / 512;                        // columns per chunk (64 or 32)
+            constexpr int RB = CW * 2, CCH = RB / 16;                  // bytes and 16-byte chunks per row
+            uint8_t* stage = smem + L::kV + (e.g_last % VST) * L::kTile + (warp - kSoftWarp0) * 32 * RB;
+            T* out = static_cast<T*>(p.out);
+#pragma unroll
+            for (int c0 = 0; c0 < HD; c0 += CW) {
+#pragma unroll
+                for (int cc = 0; cc < CCH; ++cc) {
+                    const int k = c0 / 2 + 4 * cc;
+                    *reinterpret_cast<uint4*>(stage + lane * RB + ((cc ^ (lane % CCH)) * 16)) =
+                        make_uint4(ob[k], ob[k + 1], ob[k + 2], ob[k + 3]);
+                }
+                __syncwarp();
+#pragma unroll
+                for (int it = 0; it < CCH; ++it) {
+                    const int idx = it * 32 + lane, rr = idx / CCH, cc = idx % CCH;
+                    const int tr = e.r0 + quarter * 32 + rr;              // row within the chunk
+                    const uint4 val = *reinterpret_cast<const uint4*>(stage + rr * RB + ((cc ^ (rr % CCH)) * 16));
+                    if (tr < e.n)
+                        *reinterpret_cast<uint4*>(out + (static_cast<size_t>(e.q0 + tr) * Hq + e.h0 + x) * HD + c0 +
+                                                  cc * 8) = val;
+                }
+                __syncwarp();
+            }
+            if (lane == 0) ptx::mbar_arrive(bars.stage_free(e.uc));
+            return true;
+        };
         UnitLoad ld = unit_load<NT>(p, blockIdx.x, num_units);
         for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
             const Unit w = unit_of<NT>(p, u, num_qt, ld, false);
@@ -645,60 +720,20 @@ prefill_tc_kernel(const PrefillParams p, int num_qt, const __grid_constant__ CUt
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(bars.p_full(x));       // one arrival per warp
-            }
-            if (!ok) break;
-            // epilogue: O / l -> out.  Every P.V of the unit is done once the last tile's
-            // o_full has fired (commits track all earlier MMAs), so the V stage of the
-            // unit's last key tile is free: the rows go through it, a column chunk at a
-            // time (each warp 32 rows x CW columns; 16-byte chunk c of a row at position
-            // c ^ (row % CCH), conflict-free), and leave as whole row segments.
-            ok = warp_wait(bars.o_full(NT - 1), uc & 1, lane, abort_flag, p.status);
-            if (!ok) break;
-            ptx::tc_fence_after();
-            {
-                constexpr int CW = L::kTile / 512;                   // columns per chunk (64 or 32)
-                constexpr int RB = CW * 2, CCH = RB / 16;             // bytes and 16-byte chunks per row
-                const float inv = 1.f / l;
-                uint8_t* stage = smem + L::kV + ((g - 1) % VST) * L::kTile + (warp - kSoftWarp0) * 32 * RB;
-                T* out = static_cast<T*>(p.out);
-#pragma unroll 1
-                for (int c0 = 0; c0 < HD; c0 += CW) {
-#pragma unroll
-                    for (int c = 0; c < CW / 32; ++c) {
-                        uint32_t o[32];
-                        ptx::tmem_ld32(tO + c0 + 32 * c, o);
-                        ptx::tc_wait_ld();
-                        uint32_t wv[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            wv[i] = pack2<T>(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int cc = 4 * c + i;
-                            *reinterpret_cast<uint4*>(stage + lane * RB + ((cc ^ (lane % CCH)) * 16)) =
-                                make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
-                        }
-                    }
-                    __syncwarp();
-#pragma unroll
-                    for (int it = 0; it < CCH; ++it) {
-                        const int idx = it * 32 + lane, rr = idx / CCH, cc = idx % CCH;
-                        const int tr = w.r0 + quarter * 32 + rr;          // row within the chunk
-                        const uint4 val = *reinterpret_cast<const uint4*>(stage + rr * RB + ((cc ^ (rr % CCH)) * 16));
-                        if (tr < w.n)
-                            *reinterpret_cast<uint4*>(out + (static_cast<size_t>(w.q0 + tr) * Hq + w.h0 + x) * HD + c0 +
-                                                      cc * 8) = val;
-                    }
-                    __syncwarp();
+                if (j == 0 && pending) {
+                    ok = epilogue();
+                    if (!ok) break;
+                    pending = false;
                 }
             }
-            // O is read and the staging area drained: the next unit's first P.V may overwrite
-            // O, and the V producer may refill the stage
-            ptx::tc_fence_before();
+            if (!ok) break;
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(bars.o_empty(uc));
+            if (lane == 0) *pend_s = Pending{w.q0, w.n, w.r0, w.h0, g - 1, uc};
+            l_pend = l;
+            pending = true;
             ++uc;
         }
+        if (ok && pending) epilogue();
     }
 
     ptx::tc_fence_before();
