@@ -57,17 +57,17 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by workload, with the
 # hash of the kernel sources it was taken on; reported only while they match.
 TRAFFIC = {
-    # decode_mma_kernel: 586.82 MB per launch at batch 16 (the capture-size case), 1.0091 x its
+    # decode_mma_kernel: 585.26 MB per launch at batch 16 (the capture-size case), 1.0064 x its
     # algorithmic bytes; scaled to the batch-64 launch by algorithmic bytes (2346.50 MB)
-    "llama2_7b_mha_decode": {"bytes": 2367850000, "kernel_sha": "22b9d62d2b0642b1"},
-    # decode_mma_kernel (GQA, 8 query heads per KV head): 317.67 MB per launch at batch 32 (the
-    # capture-size case), 1.012 x its algorithmic bytes; scaled to the batch-128 launch (1396.15 MB)
-    "llama2_70b_gqa_decode": {"bytes": 1412900000, "kernel_sha": "22b9d62d2b0642b1"},
-    # decode_mma_kernel (int8 codes + fp16 scales): 281.64 MB per launch at batch 1 (the capture-size
-    # case), 1.033 x its algorithmic bytes (split partials included); scaled to batch 4 (1090.59 MB)
-    "long_ctx_split_kv_int8": {"bytes": 1126600000, "kernel_sha": "22b9d62d2b0642b1"},
-    # prefill_tc_kernel: 54.66 MB read + 4.87 MB written per launch, full workload, cold L2
-    "chunked_prefill_shared_prefix": {"bytes": 59527936, "kernel_sha": "1e682f307657a38b"},
+    "llama2_7b_mha_decode": {"bytes": 2361500000, "kernel_sha": "80445fa831350776"},
+    # decode_mma_kernel (GQA, 8 query heads per KV head): 318.17 MB per launch at batch 32 (the
+    # capture-size case), 1.0136 x its algorithmic bytes; scaled to the batch-128 launch (1396.15 MB)
+    "llama2_70b_gqa_decode": {"bytes": 1415100000, "kernel_sha": "80445fa831350776"},
+    # decode_mma_kernel (int8 codes + fp16 scales): 277.87 MB per launch at batch 1 (the capture-size
+    # case), 1.0191 x its algorithmic bytes (split partials included); scaled to batch 4 (1090.59 MB)
+    "long_ctx_split_kv_int8": {"bytes": 1111500000, "kernel_sha": "80445fa831350776"},
+    # prefill_tc_kernel: 54.90 MB read + 3.79 MB written per launch, full workload, cold L2
+    "chunked_prefill_shared_prefix": {"bytes": 58690304, "kernel_sha": "8dd25261cea8f854"},
     # kv_scatter_kernel: 1120.62 MB per launch at a source batch of 16 (35 476 rows; ~43 MB of the
     # writes still in L2 at the end), scaled to the 143 153-row launch by rows
     "kv_cache_write_full": {"bytes": 4521850000, "kernel_sha": "d05e87c4610560d2"},
@@ -205,7 +205,8 @@ class L2Flush:
     def __init__(self):
         import torch
         self.wr = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-        self.rd = torch.zeros(FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
+        # float32, so that the sum reads it in place (an int32 sum would first widen a copy)
+        self.rd = torch.zeros(FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
 
     def __call__(self):
         self.wr.fill_(1)
