@@ -11,19 +11,20 @@
 // Flash Attention，让 Token 生成快 3 倍" ("Flash Attention 的分块计算原理"),
 // K/V read page by page through the block table.
 //
-// B200 design.  One CTA of 12 warps per (128-row query tile, pair of query
-// heads, sequence).  The two query heads of a pair read the same KV head
-// (grouped-query attention, "LLM推理系统优化：KV缓存管理与动态批处理技术"
-// §2.1), so they share the causal mask, the key range and every K/V tile: each
-// tile is loaded once and feeds two S tiles and two PV tiles.  The two query
-// tiles ("A" and "B") form a ping-pong: while the softmax of one runs on the
-// CUDA cores, the tensor pipe works on the other.
+// B200 design.  A persistent kernel: one CTA of 12 warps per SM walks work units
+// (128-row query tile, pair of query heads, sequence), heaviest first.  The two
+// query heads of a pair read the same KV head (grouped-query attention,
+// "LLM推理系统优化：KV缓存管理与动态批处理技术" §2.1), so they share the causal
+// mask, the key range and every K/V tile: each tile is loaded once and feeds two
+// S tiles and two PV tiles.  The two query tiles ("A" and "B") form a ping-pong:
+// while the softmax of one runs on the CUDA cores, the tensor pipe works on the
+// other.  The rings, barrier phases and key-tile count run on across units.
 //  * TMEM (512 columns): S_A | S_B | O_A | O_B, 128 columns each.  P (bf16)
 //    overwrites the first half of its own S tile.
 //  * warp 0 = K producer, warp 1 = V producer: per 128-key tile, one 16-row TMA
 //    box per page group and 64-column half (one box per lane), into rings of 3
-//    K stages and 2 V stages (mbarrier expect_tx).  Warp 0 also loads both Q
-//    tiles once.
+//    K stages and 2 V stages; one barrier per load step carries K tile t and V
+//    tile t-1.  Warp 0 also loads each unit's two Q tiles.
 //  * warp 2 = MMA issuer (one thread), per key tile j:
 //        PV_A(j)  S_A(j+1)  PV_B(j)  S_B(j+1)
 //    S = Q K^T (M=128, N=128, both operands K-major in shared memory), PV = P V
@@ -37,12 +38,14 @@
 //    FFMA, row sum, P packed to bf16 pairs and tcgen05.st over the S columns;
 //    one P-ready arrival per warp.  The accumulator is rescaled only when a
 //    row's running max grows by more than 2^8 (P <= 256 otherwise); the final
-//    division by the row sum makes any consistent reference max exact.
+//    division by the row sum makes any consistent reference max exact.  The same
+//    warps write a unit's output after the next unit's first key tile.
 //  * Heads of a group that cannot be paired (an odd group size) run one tile
-//    per CTA through the same code (NT = 1).
-//  * Every mbarrier wait polls (test_wait) and is bounded in time; on time-out
-//    the CTA records PKV_ERR_DEVICE_TIMEOUT, raises an abort flag so every role
-//    leaves its loop, waits (bounded) for its own async work and frees TMEM.
+//    per unit through the same code (NT = 1).
+//  * Every mbarrier wait is bounded in time (a waiting thread suspends in
+//    try_wait); on time-out the CTA records PKV_ERR_DEVICE_TIMEOUT, raises an
+//    abort flag so every role leaves its loop, waits (bounded) for its own async
+//    work and frees TMEM.
 #include <cuda.h>
 
 #include <cmath>
@@ -518,8 +521,16 @@ prefill_tc_kernel(const PrefillParams p, int num_qt, const __grid_constant__ CUt
             end_g[uc & 1] = g - 1;
             ++uc;
         }
-        // the step after the last tile carries no K tile
-        if (ok && is_k && lane == 0) ptx::mbar_arrive(bars.kv_full(g % KST));
+        // The step after the last tile carries no K tile.  Like a K tile, its arrival waits
+        // until the step KST back on the same barrier has been consumed (the S MMA of tile
+        // g - KST is done): otherwise it could land while that earlier step still waits for
+        // its V tile (the V warp may lag behind an epilogue's staging area) and would
+        // complete that step's phase without it.
+        if (ok && is_k) {
+            if (g >= KST)
+                ok = warp_wait(bars.s_full(NT - 1, g % KST), ((g - KST) / KST) & 1, lane, abort_flag, p.status);
+            if (ok && lane == 0) ptx::mbar_arrive(bars.kv_full(g % KST));
+        }
         if (*abort_flag && lane == 0) {
             // let the copies this warp issued land before the CTA's shared memory is released
             const int last = is_k ? g : g + 1;

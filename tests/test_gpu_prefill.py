@@ -80,6 +80,22 @@ def test_chunked_prefill_shared_prefix_full():
 
 # ---- local (sliding-window) attention ---------------------------------------------
 
+@pytest.mark.parametrize("window", [512, 128])
+def test_chunked_prefill_shared_prefix_full_window(window):
+    """The full chunked-prefill workload under local attention, in the launch shape the
+    bench times: every work unit has only a few key tiles, so a CTA walks many short units
+    (the load-step barrier's last arrival of each CTA must wait like a K tile, or it can
+    complete an earlier step's phase while the V warp still lags behind an epilogue)."""
+    c = W.chunked_prefill_shared_prefix()
+    rng = np.random.default_rng(1)
+    Hq = c.num_q_heads
+    T = c.q.shape[0]
+    items = set(rng.choice(T * Hq, 2000, replace=False).tolist())
+    for t in (0, 127, 128, 511, 512, 4095):
+        items |= {t * Hq + h for h in range(Hq)}
+    run_prefill(c, items=np.array(sorted(items)), window=window)
+
+
 @pytest.mark.parametrize("window", [1, 64, 128, 129, 300])
 def test_sliding_window_prefill(window):
     run_prefill(case(20, chunks=(1, 5, 64, 130, 200, 128), private_prefix=7, shared_prefix=256), window=window)
