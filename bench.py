@@ -67,7 +67,7 @@ TRAFFIC = {
     # case), 1.0191 x its algorithmic bytes (split partials included); scaled to batch 4 (1090.59 MB)
     "long_ctx_split_kv_int8": {"bytes": 1111500000, "kernel_sha": "80445fa831350776"},
     # prefill_tc_kernel: 54.90 MB read + 3.79 MB written per launch, full workload, cold L2
-    "chunked_prefill_shared_prefix": {"bytes": 58690304, "kernel_sha": "8dd25261cea8f854"},
+    "chunked_prefill_shared_prefix": {"bytes": 58690304, "kernel_sha": "c57d9dcdfe3ec513"},
     # kv_scatter_kernel: 1120.62 MB per launch at a source batch of 16 (35 476 rows; ~43 MB of the
     # writes still in L2 at the end), scaled to the 143 153-row launch by rows
     "kv_cache_write_full": {"bytes": 4521850000, "kernel_sha": "d05e87c4610560d2"},
@@ -451,8 +451,8 @@ class GraphStep:
     def __init__(self, inner):
         from paged_kv_cache_380_b200.graph import DecodeStepGraph
         self.inner = inner
-        for k in ("case", "kind", "int8", "has_new", "decode_bytes", "write_bytes", "work", "units", "launches",
-                  "splits", "split_tokens"):
+        for k in ("case", "kind", "int8", "window", "has_new", "decode_bytes", "write_bytes", "work", "units",
+                  "launches", "splits", "split_tokens"):
             setattr(self, k, getattr(inner, k))
         kw = dict(k_scales=inner.ks, v_scales=inner.vs)
         if inner.has_new:
@@ -542,52 +542,71 @@ def cpu_baseline(step, budget_s: float = 20.0):
         return {"value": rate / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
                 "sample": f"all {T} rows of the scatter, one row copy each ({dt:.2f} s)", "seconds": dt}
     if step.kind == "decode":
-        B = c.batch
-        total_ctx = c.context_lens.astype(np.int64).sum()
+        B, Hq = c.batch, c.num_q_heads
+        eff = c.context_lens.astype(np.int64)
+        if getattr(step, "window", 0) > 0:
+            eff = np.minimum(eff, step.window)                 # keys a windowed query reads
+        _oracle_inputs(step)                                   # untimed: the appended / quantised pool
 
         def sample(n_threads, seconds):
-            # the first S sequences (all heads), S sized to ~seconds from a 1-sequence probe
+            # the first S sequences (all heads), S grown until the run takes about `seconds`
             oracle.set_threads(n_threads)
             try:
-                t0 = time.perf_counter()
-                _run_oracle_decode(step, np.arange(c.num_q_heads))
-                one = max(time.perf_counter() - t0, 1e-3)
-                S = int(max(1, min(B, seconds / one)))
-                t0 = time.perf_counter()
-                _run_oracle_decode(step, np.arange(S * c.num_q_heads))
-                dt = time.perf_counter() - t0
+                S, dt, reps = 1, 0.0, 1
+                for _ in range(5):
+                    t0 = time.perf_counter()
+                    _run_oracle_decode(step, np.arange(S * Hq))
+                    dt = time.perf_counter() - t0
+                    if dt >= seconds / 2 or S == B:
+                        break
+                    S = int(min(B, max(S + 1, S * seconds / max(dt, 1e-3))))
+                if dt < seconds / 2:                           # the whole batch is quicker: repeat it
+                    reps = int(min(20, np.ceil(seconds / 2 / max(dt, 1e-3))))
+                    t0 = time.perf_counter()
+                    for _ in range(reps):
+                        _run_oracle_decode(step, np.arange(S * Hq))
+                    dt = time.perf_counter() - t0
             finally:
                 oracle.set_threads(threads)
-            work = step.decode_bytes * c.context_lens[:S].astype(np.int64).sum() / total_ctx
-            return work / dt / 1e9, S, dt
+            work = reps * step.decode_bytes * eff[:S].sum() / eff.sum()
+            return work / dt / 1e9, (S if reps == 1 else f"{S} (x{reps})"), dt
 
         v, S, dt = sample(threads, budget_s / 2)
         v1, S1, dt1 = sample(1, budget_s / 4)
         return {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle",
-                "sample": f"decode of the first {S} of {B} sequences, all {c.num_q_heads} heads, fp64 "
-                          f"({dt:.1f} s)", "seconds": dt,
+                "sample": f"decode of the first {S} of {B} sequences, all {Hq} heads, fp64 ({dt:.1f} s)",
+                "seconds": dt,
                 "single_thread": {"value": v1, "unit": "GB/s", "cores": 1,
                                   "sample": f"decode of the first {S1} of {B} sequences, all heads, fp64, "
                                             f"one thread ({dt1:.1f} s)"}}
     T = c.q.shape[0]
     Hq = c.num_q_heads
     rng = np.random.default_rng(0)
+    _oracle_inputs(step)
 
     def sample(n_threads, seconds):
-        # random (row, head) items, their number sized to ~seconds from a 64-item probe
+        # random (row, head) items, their number grown until the run takes about `seconds`
         oracle.set_threads(n_threads)
         try:
-            t0 = time.perf_counter()
-            _run_oracle_prefill(step, rng.choice(T * Hq, 64, replace=False))
-            per = max((time.perf_counter() - t0) / 64, 1e-6)
-            n = int(min(T * Hq, max(64, seconds / per)))
-            items = rng.choice(T * Hq, n, replace=False)
-            t0 = time.perf_counter()
-            _run_oracle_prefill(step, items)
-            dt = time.perf_counter() - t0
+            n, dt, reps = 64, 0.0, 1
+            for _ in range(5):
+                items = rng.choice(T * Hq, n, replace=False)
+                t0 = time.perf_counter()
+                _run_oracle_prefill(step, items)
+                dt = time.perf_counter() - t0
+                if dt >= seconds / 2 or n == T * Hq:
+                    break
+                n = int(min(T * Hq, max(n + 1, n * seconds / max(dt, 1e-3))))
+            if dt < seconds / 2:                               # every item is quicker: repeat them
+                reps = int(min(20, np.ceil(seconds / 2 / max(dt, 1e-3))))
+                t0 = time.perf_counter()
+                for _ in range(reps):
+                    _run_oracle_prefill(step, items)
+                dt = time.perf_counter() - t0
         finally:
             oracle.set_threads(threads)
-        return step.work * n / (T * Hq) / dt / 1e12, n, dt
+        # items are drawn uniformly, so their share of the flops is their share of the items
+        return reps * step.work * n / (T * Hq) / dt / 1e12, (n if reps == 1 else f"{n} (x{reps})"), dt
 
     v, n, dt = sample(threads, budget_s / 2)
     v1, n1, dt1 = sample(1, budget_s / 4)
@@ -598,29 +617,40 @@ def cpu_baseline(step, budget_s: float = 20.0):
                                         f"({dt1:.1f} s)"}}
 
 
+def _oracle_inputs(step):
+    """The pool the oracle reads (after the step's cache append, or quantised for INT8),
+    built once per step object outside any timed region."""
+    import oracle
+    if hasattr(step, "_oracle_kv"):
+        return step._oracle_kv
+    c = step.case
+    if getattr(step, "int8", False):
+        kq, ks = oracle.quantize_int8(c.k_pages, c.dtype)
+        vq, vs = oracle.quantize_int8(c.v_pages, c.dtype)
+        step._oracle_kv = (kq, vq, "i8", ks, vs)
+    else:
+        k, v = c.k_pages, c.v_pages
+        if c.k_new is not None and c.slot_mapping is not None and len(c.slot_mapping):
+            k, v = k.copy(), v.copy()
+            oracle.kv_cache_write(c.k_new, c.v_new, c.slot_mapping, k, v)
+        step._oracle_kv = (k, v, c.dtype, None, None)
+    return step._oracle_kv
+
+
 def _run_oracle_decode(step, items):
     import oracle
     c = step.case
-    if step.int8:
-        if not hasattr(step, "_q8"):
-            step._q8 = (*oracle.quantize_int8(c.k_pages, c.dtype), *oracle.quantize_int8(c.v_pages, c.dtype))
-        kq, ks, vq, vs = step._q8
-        return oracle.decode(c.q, c.dtype, kq, vq, "i8", c.block_tables, c.context_lens, c.scale,
-                             k_scales=ks, v_scales=vs, items=items)
-    k, v = c.k_pages, c.v_pages
-    if step.has_new:
-        k, v = k.copy(), v.copy()
-        oracle.kv_cache_write(c.k_new, c.v_new, c.slot_mapping, k, v)
-    return oracle.decode(c.q, c.dtype, k, v, c.dtype, c.block_tables, c.context_lens, c.scale, items=items)
+    k, v, kv_tag, ks, vs = _oracle_inputs(step)
+    return oracle.decode(c.q, c.dtype, k, v, kv_tag, c.block_tables, c.context_lens, c.scale,
+                         k_scales=ks, v_scales=vs, items=items, window=getattr(step, "window", 0))
 
 
 def _run_oracle_prefill(step, items):
     import oracle
     c = step.case
-    k, v = c.k_pages.copy(), c.v_pages.copy()
-    oracle.kv_cache_write(c.k_new, c.v_new, c.slot_mapping, k, v)
-    return oracle.prefill(c.q, c.dtype, k, v, c.dtype, c.block_tables, c.q_start, c.context_lens, True,
-                          c.scale, items=items)
+    k, v, kv_tag, _, _ = _oracle_inputs(step)
+    return oracle.prefill(c.q, c.dtype, k, v, kv_tag, c.block_tables, c.q_start, c.context_lens, True,
+                          c.scale, items=items, window=getattr(step, "window", 0))
 
 
 def run_ours(args):
