@@ -36,7 +36,8 @@
 //    lane (query row) per thread, all 128 columns of its row.  tcgen05.ld of
 //    the S row, masking, row max, 2^(s*scale - m) with the scale folded into one
 //    FFMA, row sum, P packed to bf16 pairs and tcgen05.st over the S columns;
-//    one P-ready arrival per warp.  The accumulator is rescaled only when a
+//    one arrival per warp when the first 64 keys' P is stored (P.V over them
+//    starts while the other 64 are computed) and one when all of P is.  The accumulator is rescaled only when a
 //    row's running max grows by more than 2^8 (P <= 256 otherwise); the final
 //    division by the row sum makes any consistent reference max exact.  The same
 //    warps write a unit's output after the next unit's first key tile.
@@ -77,7 +78,7 @@ struct Layout {
     static constexpr int kK = kQ + NT * kTile;
     static constexpr int kV = kK + KST * kTile;
     static constexpr int kBar = kV + VST * kTile;
-    static constexpr int kNumBars = 23;
+    static constexpr int kNumBars = 25;
     static constexpr int kPend = kBar + kNumBars * 8 + 16;  // after the TMEM address and abort flag
     static constexpr int kEnd = kPend + 8 * 32;             // a pending epilogue's unit, per softmax warp
     // The CTA holds all of TMEM, so only one may run per SM: ask for more than
@@ -104,8 +105,10 @@ struct Bars {
     // alternate by unit parity so that a waiter one unit behind is never two phases late
     __device__ __forceinline__ uint32_t o_read(int uc) const { return at(6 + 3 * KST + 2 * VST + (uc & 1)); }
     __device__ __forceinline__ uint32_t stage_free(int uc) const { return at(8 + 3 * KST + 2 * VST + (uc & 1)); }
+    // P of tile x's first 64 keys is in place (P.V over them may start); phase per key tile
+    __device__ __forceinline__ uint32_t p_half(int x) const { return at(10 + 3 * KST + 2 * VST + x); }
 };
-static_assert(8 + 3 * KST + 2 * VST + 2 == 23, "barrier count");
+static_assert(10 + 3 * KST + 2 * VST + 2 == 25, "barrier count");
 
 // sm_100 shared-memory matrix descriptor: start, leading and stride byte
 // offsets (>> 4), version 1, SWIZZLE_128B layout.
@@ -343,19 +346,23 @@ struct Issuer {
         }
         ptx::tc_commit(bars.s_full(x, ks));
     }
-    // O_x (+)= P_x V[stage vs]; the first key tile of a unit overwrites O.
-    __device__ __forceinline__ void pv(int x, int vs, bool acc) const {
+    // O_x (+)= P_x V[stage vs] over keys 64 h .. 64 h + 63; the first key tile of a unit
+    // overwrites O.
+    __device__ __forceinline__ void pv(int x, int vs, bool acc, int h) const {
         constexpr uint32_t id = idesc_f16<T>(BM, HD, 1);
         const uint64_t b = dv + static_cast<uint64_t>((vs * L::kTile) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
+        for (int k = 0; k < BN / 32; ++k) {
+            const int kk = h * (BN / 32) + k;
             ptx::tc_mma_ts(kOCol + x * 128, static_cast<uint32_t>(x * 128 + kk * 8), b + static_cast<uint64_t>((kk * 2048) >> 4),
                            id, (acc || kk > 0) ? 1u : 0u);
+        }
     }
     // One unit of n key tiles, global tiles g0 .. g0+n-1: S_A(0) [S_B(0)], then per key
-    // tile j: PV_A(j) S_A(j+1) [PV_B(j) S_B(j+1)].  Three barrier probes per key tile (the
-    // K/V step, P_A, P_B): each probe costs the tensor pipe about as much as two MMAs when
-    // nothing is queued behind it.
+    // tile j: PV_A(j) S_A(j+1) [PV_B(j) S_B(j+1)], each PV in two halves of 64 keys released
+    // by their own barrier.  Five barrier probes per key tile (the K/V step, then each
+    // half of P_A and of P_B): each probe costs the tensor pipe about as much as two MMAs
+    // when nothing is queued behind it.
     // uc = units this CTA has issued before (the Q, O-ready and O-read barriers' phase).
     __device__ bool unit(int g0, int n, int uc) const {
         if (!wait(bars.q_full(), uc & 1)) return false;
@@ -371,16 +378,23 @@ struct Issuer {
             if (!wait(bars.kv_full(ks1), ((g + 1) / KST) & 1)) return false;
             // the unit's first P.V overwrites O: the previous unit's epilogue must have read it
             if (j == 0 && uc > 0 && !wait(bars.o_read(uc - 1), ((uc - 1) >> 1) & 1)) return false;
+            // P.V over a tile's first 64 keys starts while its softmax finishes the other 64
+            if (!wait(bars.p_half(0), g & 1)) return false;
+            ptx::tc_fence_after();
+            pv(0, vs, j > 0, 0);
             if (!wait(bars.p_full(0), g & 1)) return false;
             ptx::tc_fence_after();
-            pv(0, vs, j > 0);
+            pv(0, vs, true, 1);
             if (NT == 1) ptx::tc_commit(bars.pv_done(vs));
             if (!more) ptx::tc_commit(bars.o_full(0));
             if (more) s(0, ks1);
             if (NT == 2) {
+                if (!wait(bars.p_half(1), g & 1)) return false;
+                ptx::tc_fence_after();
+                pv(1, vs, j > 0, 0);
                 if (!wait(bars.p_full(1), g & 1)) return false;
                 ptx::tc_fence_after();
-                pv(1, vs, j > 0);
+                pv(1, vs, true, 1);
                 ptx::tc_commit(bars.pv_done(vs));
                 if (!more) ptx::tc_commit(bars.o_full(1));
                 if (more) s(1, ks1);
@@ -419,6 +433,7 @@ prefill_tc_kernel(const PrefillParams p, int num_qt, const __grid_constant__ CUt
         for (int i = 0; i < VST; ++i) ptx::mbar_init(bars.pv_done(i), 1);
         for (int x = 0; x < 2; ++x) {
             ptx::mbar_init(bars.p_full(x), 4);                  // one arrival per softmax warp
+            ptx::mbar_init(bars.p_half(x), 4);
             ptx::mbar_init(bars.o_full(x), 1);
             ptx::mbar_init(bars.o_read(x), 4 * NT);             // one arrival per softmax warp
             ptx::mbar_init(bars.stage_free(x), 4 * NT);
@@ -688,6 +703,22 @@ prefill_tc_kernel(const PrefillParams p, int num_qt, const __grid_constant__ CUt
                         ptx::tmem_st16(tO + 16 * c, o);
                     }
                 }
+                if (x == 0 && w.ctx < (jt + 1) * BN) {
+                    // V rows past the context (tail of the last page, or never loaded) must be
+                    // finite zeros: P is 0 there but 0 * NaN would poison O.  Tile A's warps do it
+                    // before either half of P_A(j) is released (PV_A(j) runs before PV_B(j)).
+                    const int vs = g % VST;
+                    ok = warp_wait(bars.kv_full((g + 1) % KST), ((g + 1) / KST) & 1, lane, abort_flag, p.status);
+                    if (!ok) break;
+                    const int first = w.ctx - jt * BN;                  // first invalid row of the tile
+                    uint4* vt = reinterpret_cast<uint4*>(smem + L::kV + vs * L::kTile);
+                    const int tid = threadIdx.x - kSoftWarp0 * 32, per = (BN - first) * 8;
+                    for (int idx = tid; idx < L::NH * per; idx += 128) {
+                        const int a = idx / per, rem = idx % per;
+                        vt[(a * kAtom + (first + rem / 8) * 128) / 16 + rem % 8] = make_uint4(0, 0, 0, 0);
+                    }
+                    ptx::fence_proxy_async_smem();
+                }
                 const float neg = m_ref == -INFINITY ? 0.f : -m_ref;      // no key seen yet: all p are 0
                 // one packed FMA per key pair, one SFU exponential per key
                 const uint64_t sc2 = f2pack(sl2, sl2), ng2 = f2pack(neg, neg);
@@ -704,6 +735,13 @@ prefill_tc_kernel(const PrefillParams p, int num_qt, const __grid_constant__ CUt
                     // P column c holds keys 2c, 2c+1: half hh goes to columns 32 hh .. 32 hh + 31,
                     // which hold scores this thread has already read
                     tmem_st32(tS + 32 * hh, pk);
+                    if (hh == 0) {
+                        // the first 64 keys' P is in place: P.V over them may start
+                        ptx::tc_wait_st();
+                        ptx::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(bars.p_half(x));
+                    }
                 }
                 {
                     float a0, a1, b0, b1;
@@ -712,22 +750,6 @@ prefill_tc_kernel(const PrefillParams p, int num_qt, const __grid_constant__ CUt
                     l += (a0 + a1) + (b0 + b1);
                 }
                 ptx::tc_wait_st();
-                if (x == 0 && w.ctx < (jt + 1) * BN) {
-                    // V rows past the context (tail of the last page, or never loaded) must be
-                    // finite zeros: P is 0 there but 0 * NaN would poison O.  Tile A's warps do it
-                    // before PV_A(j), which runs before PV_B(j).
-                    const int vs = g % VST;
-                    ok = warp_wait(bars.kv_full((g + 1) % KST), ((g + 1) / KST) & 1, lane, abort_flag, p.status);
-                    if (!ok) break;
-                    const int first = w.ctx - jt * BN;                  // first invalid row of the tile
-                    uint4* vt = reinterpret_cast<uint4*>(smem + L::kV + vs * L::kTile);
-                    const int tid = threadIdx.x - kSoftWarp0 * 32, per = (BN - first) * 8;
-                    for (int idx = tid; idx < L::NH * per; idx += 128) {
-                        const int a = idx / per, rem = idx % per;
-                        vt[(a * kAtom + (first + rem / 8) * 128) / 16 + rem % 8] = make_uint4(0, 0, 0, 0);
-                    }
-                    ptx::fence_proxy_async_smem();
-                }
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(bars.p_full(x));       // one arrival per warp

@@ -64,10 +64,8 @@ def roles_for(units, NT):
                 if j == 0 and uc > 0:
                     yield ("wait", ("o_read", (uc - 1) & 1), (uc - 1) >> 1)
                 for x in range(NT):
-                    if x == 1:
-                        yield ("wait", ("p_full", 1), gg)
-                    else:
-                        yield ("wait", ("p_full", 0), gg)
+                    yield ("wait", ("p_half", x), gg)
+                    yield ("wait", ("p_full", x), gg)
                     if x == NT - 1:
                         yield ("arrive", ("pv_done", vs), gg // VST)
                     if not more:
@@ -89,6 +87,7 @@ def roles_for(units, NT):
         for n_tiles in units:
             for j in range(n_tiles):
                 yield ("wait", ("s_full", x, g % KST), g // KST)
+                yield ("arrive", ("p_half", x), g)
                 yield ("arrive", ("p_full", x), g)
                 if j == 0 and pending is not None:
                     yield from epilogue(pending)
@@ -103,7 +102,7 @@ def roles_for(units, NT):
     for x in range(NT):
         for w in range(4):
             roles[f"S{x}{w}"] = softmax(x)
-    counts = {"q_full": 1, "kv_full": 2, "s_full": 1, "p_full": 4, "pv_done": 1, "o_full": 1,
+    counts = {"q_full": 1, "kv_full": 2, "s_full": 1, "p_full": 4, "p_half": 4, "pv_done": 1, "o_full": 1,
               "o_read": 4 * NT, "stage_free": 4 * NT}
     return roles, counts
 
