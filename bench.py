@@ -66,8 +66,8 @@ TRAFFIC = {
     # decode_mma_kernel (int8 codes + fp16 scales): 277.87 MB per launch at batch 1 (the capture-size
     # case), 1.0191 x its algorithmic bytes (split partials included); scaled to batch 4 (1090.59 MB)
     "long_ctx_split_kv_int8": {"bytes": 1111500000, "kernel_sha": "80445fa831350776"},
-    # prefill_tc_kernel: 54.92 MB read + 4.19 MB written per launch, full workload, cold L2
-    "chunked_prefill_shared_prefix": {"bytes": 59116544, "kernel_sha": "38da3c05edf0bfae"},
+    # prefill_tc_kernel: 54.76 MB read + 3.63 MB written per launch, full workload, cold L2
+    "chunked_prefill_shared_prefix": {"bytes": 58394112, "kernel_sha": "19f948ac33e1e7cf"},
     # kv_scatter_kernel: 1120.62 MB per launch at a source batch of 16 (35 476 rows; ~43 MB of the
     # writes still in L2 at the end), scaled to the 143 153-row launch by rows
     "kv_cache_write_full": {"bytes": 4521850000, "kernel_sha": "d05e87c4610560d2"},

@@ -6,8 +6,9 @@ the library a scratch buffer on demand (a server that reserved all HBM for
 its KV-cache pool at start-up, a plain-C host without a device allocator, a
 decode loop that must not risk a synchronising allocation).  Here it is
 called through the C ABI twice in a row, with different problems, and must
-agree with the workspace entry point within the bf16 tolerance (2e-2); a
-problem needing more scratch than the array holds is refused before launch.
+agree with the fp64 oracle and with the workspace entry point within the
+bf16 tolerance (2e-2); a problem needing more scratch than the array holds
+is refused before launch.
 
 This file is named to be collected last, and passes alone in a fresh process
 as well as after the other tests.
@@ -18,7 +19,8 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_util import assert_status_ok, dev, f64
+import oracle
+from gpu_util import assert_close, assert_status_ok, dev, f64
 from paged_kv_cache_380_b200 import ops
 from paged_kv_cache_380_b200 import workloads as W
 
@@ -66,6 +68,13 @@ def test_noalloc_decode_matches_workspace_decode_on_two_calls():
         g, w = f64(got), f64(want)
         assert np.isfinite(g).all()
         assert np.max(np.abs(g - w)) <= 2e-2
+        # and against the oracle: every (sequence, head) of the small problem, a sample of the large one
+        n_items = c.batch * c.num_q_heads
+        items = (np.arange(n_items) if call == 0 else
+                 np.sort(np.random.default_rng(3).choice(n_items, 256, replace=False)))
+        ref = oracle.decode(c.q, "bf16", c.k_pages, c.v_pages, "bf16", c.block_tables, c.context_lens, c.scale,
+                            items=items)
+        assert_close(g.reshape(n_items, -1)[items], ref, 2e-2, c.name)
 
 
 def test_noalloc_decode_refuses_problems_beyond_the_scratch():
