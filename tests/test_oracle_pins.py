@@ -368,7 +368,9 @@ def test_f16_widening_and_rounding_match_numpy():
     x = np.concatenate([rng.standard_normal(4000).astype(np.float32) * 10.0 ** rng.integers(-9, 6, 4000),
                         np.array([65504, 65519.99, 65520, 1e-8, 2.0 ** -24, 2.0 ** -25,
                                   3 * 2.0 ** -26, 6.1e-5, -0.0, 0.0], dtype=np.float32)]).astype(np.float32)
-    assert np.array_equal(oracle.float_to_f16_bits(x), x.astype(np.float16).view(np.uint16))
+    with np.errstate(over="ignore"):          # values past the fp16 range round to inf on purpose
+        want = x.astype(np.float16).view(np.uint16)
+    assert np.array_equal(oracle.float_to_f16_bits(x), want)
 
 
 def test_quantiser_bounds_and_symmetry():
