@@ -63,11 +63,15 @@ struct Plan {
 
 // Split-KV partitioner.  Partitions are whole 16-token chunks (and whole pages
 // when a page holds several chunks).  Automatic choice: partitions of at most
-// 2048 tokens, shortened down to 256 tokens while the grid would otherwise not
-// fill two waves of the SMs.  The ceiling is a measured balance: longer
-// partitions mean fewer CTAs (less per-CTA set-up, fewer partials to merge) but
-// a longer tail; 2048 beat both 1024 and 4096 on every decode workload tried
-// (Llama-2-7B/70B shapes, 131k-token contexts in bf16 and INT8).
+// 2048 tokens, halved while the grid would hold fewer than 12 CTAs per SM, but
+// not below 512 tokens unless it would not even fill one wave (3 CTAs per SM),
+// and never below 256.  The numbers are measured balances: longer partitions
+// mean fewer CTAs (less per-CTA set-up, fewer partials to merge) but a longer
+// tail.  The 2048-token ceiling beat both 1024 and 4096 on every bench decode
+// workload (Llama-2-7B/70B shapes, 131k-token contexts in bf16 and INT8), which
+// the fill rule leaves untouched; at batch 16 of the Llama-2-7B shapes the
+// 12-per-SM target (1024-token partitions) is 6% faster than stopping at two
+// waves of two, and at batch 4 256-token partitions lose 2.7% against 512.
 Plan plan_decode(int num_seqs, int num_kv_heads, int page_size, int max_pages_per_seq,
                  pkv_dtype kv_dtype, int num_splits) {
     const int64_t max_tokens = static_cast<int64_t>(max_pages_per_seq) * page_size;
@@ -79,9 +83,13 @@ Plan plan_decode(int num_seqs, int num_kv_heads, int page_size, int max_pages_pe
         cps = (max_chunks + s - 1) / s;
     } else {
         const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads;
-        const int64_t want = 2LL * sm_count() * 2;   // two waves of two resident CTAs per SM
+        const int64_t sms = sm_count();
         cps = PKV_SPLIT_MAX_CHUNKS;
-        while (cps > 16 && units * ((max_chunks + cps - 1) / cps) < want) cps /= 2;
+        for (;;) {
+            const int64_t ctas = units * ((max_chunks + cps - 1) / cps);
+            if (!((cps > 32 && ctas < 12 * sms) || (cps > 16 && ctas < 3 * sms))) break;
+            cps /= 2;
+        }
     }
     const int page_chunks = page_size / kChunk > 1 ? page_size / kChunk : 1;
     cps = (cps + page_chunks - 1) / page_chunks * page_chunks;
