@@ -57,15 +57,15 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by workload, with the
 # hash of the kernel sources it was taken on; reported only while they match.
 TRAFFIC = {
-    # decode_mma_kernel: 585.26 MB per launch at batch 16 (the capture-size case), 1.0064 x its
-    # algorithmic bytes; scaled to the batch-64 launch by algorithmic bytes (2346.50 MB)
-    "llama2_7b_mha_decode": {"bytes": 2361500000, "kernel_sha": "80445fa831350776"},
-    # decode_mma_kernel (GQA, 8 query heads per KV head): 318.17 MB per launch at batch 32 (the
-    # capture-size case), 1.0136 x its algorithmic bytes; scaled to the batch-128 launch (1396.15 MB)
-    "llama2_70b_gqa_decode": {"bytes": 1415100000, "kernel_sha": "80445fa831350776"},
-    # decode_mma_kernel (int8 codes + fp16 scales): 277.87 MB per launch at batch 1 (the capture-size
-    # case), 1.0191 x its algorithmic bytes (split partials included); scaled to batch 4 (1090.59 MB)
-    "long_ctx_split_kv_int8": {"bytes": 1111500000, "kernel_sha": "80445fa831350776"},
+    # decode_mma_kernel: 1205.20 MB per launch at batch 32 (the capture-size case, same partitions
+    # as the bench launch), 1.0039 x its algorithmic bytes; scaled to batch 64 (2346.50 MB)
+    "llama2_7b_mha_decode": {"bytes": 2355600000, "kernel_sha": "96e1f88fb35756e9"},
+    # decode_mma_kernel (GQA, 8 query heads per KV head): 694.20 MB per launch at batch 64 (same
+    # partitions as the bench launch), 1.0079 x its algorithmic bytes; scaled to batch 128 (1396.15 MB)
+    "llama2_70b_gqa_decode": {"bytes": 1407200000, "kernel_sha": "96e1f88fb35756e9"},
+    # decode_mma_kernel (int8 codes + fp16 scales): the bench launch itself, 1098.35 MB (1.0071 x its
+    # algorithmic bytes, split partials included)
+    "long_ctx_split_kv_int8": {"bytes": 1098350000, "kernel_sha": "96e1f88fb35756e9"},
     # prefill_tc_kernel: 54.76 MB read + 3.63 MB written per launch, full workload, cold L2
     "chunked_prefill_shared_prefix": {"bytes": 58394112, "kernel_sha": "19f948ac33e1e7cf"},
     # kv_scatter_kernel: 1120.62 MB per launch at a source batch of 16 (35 476 rows; ~43 MB of the
