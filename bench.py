@@ -714,7 +714,9 @@ def run_ours(args):
         peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
         achieved = dom_work / (dom_avg_ms / 1e3) / 1e12
         bound, runit = "tensor", "TFLOP/s"
-    tr = TRAFFIC.get(config_key(args.workload))
+    # the ncu figures belong to the bench launch of each workload: not to other batch sizes,
+    # a local window or the graph replay
+    tr = TRAFFIC.get(config_key(args.workload)) if not (args.batch or args.window or args.graph) else None
     traffic = tr["bytes"] if tr and tr["kernel_sha"] == kernel_sha(step.kind) else None
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world, "steps": K, "warmup": W,
