@@ -57,6 +57,11 @@ def test_split_planner_on_the_workloads(lib):
     # few (sequence, head) units -> shorter partitions, never below 256 tokens
     s, t = ops.decode_plan(1, 8, 1, 128, 16, 64)
     assert t == 256 and s == 4
+    # Llama-2-7B shapes at smaller batches (148 SMs): halved while under 12 CTAs per SM, kept at
+    # 512 tokens or more while the grid fills a wave (3 CTAs per SM)
+    assert ops.decode_plan(16, 32, 32, 128, 16, 256) == (4, 1024)
+    assert ops.decode_plan(4, 32, 32, 128, 16, 256) == (8, 512)
+    assert ops.decode_plan(1, 32, 32, 128, 16, 256) == (16, 256)
     # explicit split count, and fp32 never splits
     assert ops.decode_plan(2, 4, 2, 64, 16, 7, num_splits=3)[0] == 3
     assert ops.decode_plan(2, 4, 2, 64, 16, 7, torch.float32) == (1, 112)
