@@ -5,10 +5,18 @@ tiles) is written as the sequence of waits and arrivals the kernel performs, wit
 phase each one means.  Arrivals count toward a barrier's current phase, as on the GPU, so
 an arrival that lands before the previous phase of its barrier has completed is reported
 (it would complete the wrong phase), and so is a wait whose barrier is two phases ahead
-(a parity wait could not tell them apart).  The roles are run under several scheduling
-orders; every one must finish.  The model caught the K producer's final arrival ("no K
-tile after the last one") landing in an earlier phase of its load-step barrier when short
-units (local attention) let the V producer lag behind an epilogue's staging area."""
+(a parity wait could not tell them apart).  Buffer reuse is checked too: before a K or V
+stage or the Q buffers are refilled, every query tile's S or P.V that read them must have
+been signalled, and a unit's epilogue (which stages its output in the V stage of the unit's
+last key tile) needs every tile's last P.V; a role states such a need as a "require" event,
+checked when the role reaches it.  A commit signals, with its barrier's phase, every MMA the
+issuing thread issued before it (tcgen05 MMAs of one thread complete in issue order).  The
+roles run under fixed orders (each role as far as it can go, in turn) and under random
+schedules (one operation at a time of a role picked at random), so that any role may fall
+far behind the others; every run must finish.  The model caught the K producer's final
+arrival ("no K tile after the last one") landing in an earlier phase of its load-step
+barrier when short units (local attention) let the V producer lag behind an epilogue's
+staging area."""
 import random
 
 import pytest
@@ -28,16 +36,20 @@ def roles_for(units, NT):
                 if uc > 0:
                     gl = g - 1
                     yield ("wait", ("s_full", NT - 1, gl % KST), gl // KST)
+                    yield ("require", [("S", x, gl) for x in range(NT)], None)
                 yield ("arrive", ("q_full",), uc)
             for _ in range(n_tiles):
                 st = g % nst
                 if g >= nst:
                     prev = g - nst
+                    # one issuer, in order: the last tile's S (PV) done means every tile's is
                     yield ("wait", ("s_full", NT - 1, st) if is_k else ("pv_done", st), prev // nst)
                     for e in range(2):
                         if not is_k and end_g[e] == prev:
                             ue = uc - 1 - ((uc - 1 - e) & 1)
                             yield ("wait", ("stage_free", ue & 1), ue >> 1)
+                if g >= nst:
+                    yield ("require", [("S" if is_k else "PV", x, g - nst) for x in range(NT)], None)
                 step = g if is_k else g + 1
                 yield ("arrive", ("kv_full", step % KST), step // KST)
                 g += 1
@@ -49,14 +61,23 @@ def roles_for(units, NT):
             yield ("arrive", ("kv_full", g % KST), g // KST)
 
     def issuer():
+        # one thread issues both tiles' MMAs; they complete in issue order, so a commit's
+        # barrier phase also signals every MMA issued before it
         g = uc = 0
+        issued = []
+
+        def commit(bar, phase, ev=None):
+            evs = issued + ([ev] if ev else [])
+            issued.clear()
+            return ("arrive", bar, phase, evs)
+
         for n_tiles in units:
             g0 = g
             yield ("wait", ("q_full",), uc)
             if g0 == 0:
                 yield ("wait", ("kv_full", 0), 0)
             for x in range(NT):
-                yield ("arrive", ("s_full", x, g0 % KST), g0 // KST)
+                yield commit(("s_full", x, g0 % KST), g0 // KST, ("S", x, g0))
             for j in range(n_tiles):
                 gg, more = g0 + j, j + 1 < n_tiles
                 vs, ks1 = gg % VST, (gg + 1) % KST
@@ -66,12 +87,13 @@ def roles_for(units, NT):
                 for x in range(NT):
                     yield ("wait", ("p_half", x), gg)
                     yield ("wait", ("p_full", x), gg)
+                    issued.append(("PV", x, gg))
                     if x == NT - 1:
-                        yield ("arrive", ("pv_done", vs), gg // VST)
+                        yield commit(("pv_done", vs), gg // VST)
                     if not more:
-                        yield ("arrive", ("o_full", x), uc)
+                        yield commit(("o_full", x), uc)
                     if more:
-                        yield ("arrive", ("s_full", x, ks1), (gg + 1) // KST)
+                        yield commit(("s_full", x, ks1), (gg + 1) // KST, ("S", x, gg + 1))
             g += n_tiles
             uc += 1
 
@@ -79,8 +101,9 @@ def roles_for(units, NT):
         g = uc = 0
         pending = None
 
-        def epilogue(e_uc):
+        def epilogue(e_uc, g_last):
             yield ("wait", ("o_full", NT - 1), e_uc)
+            yield ("require", [("PV", y, g_last) for y in range(NT)], None)
             yield ("arrive", ("o_read", e_uc & 1), e_uc >> 1)
             yield ("arrive", ("stage_free", e_uc & 1), e_uc >> 1)
 
@@ -90,13 +113,13 @@ def roles_for(units, NT):
                 yield ("arrive", ("p_half", x), g)
                 yield ("arrive", ("p_full", x), g)
                 if j == 0 and pending is not None:
-                    yield from epilogue(pending)
+                    yield from epilogue(*pending)
                     pending = None
                 g += 1
-            pending = uc
+            pending = (uc, g - 1)
             uc += 1
         if pending is not None:
-            yield from epilogue(pending)
+            yield from epilogue(*pending)
 
     roles = {"K": producer(True), "V": producer(False), "MMA": issuer()}
     for x in range(NT):
@@ -107,37 +130,63 @@ def roles_for(units, NT):
     return roles, counts
 
 
-def run(units, NT, order):
+def run(units, NT, order=None, rng=None):
+    """Run the roles to the end: with `order`, each role in turn as far as it can go; with
+    `rng`, one operation at a time of a role picked at random among those that can proceed
+    (so any role may fall arbitrarily far behind the others)."""
     roles, counts = roles_for(units, NT)
-    names = order(list(roles))
+    names = list(roles) if order is None else order(list(roles))
     done, pend = {}, {}
+    signalled, pend_ev = set(), {}     # events ("S"/"PV", tile x, key tile) whose barrier phase completed
     cur = {r: next(roles[r], None) for r in names}
-    progress = True
-    while progress:
-        progress = False
-        for r in names:
-            while cur[r] is not None:
-                op, bar, idx = cur[r]
-                c = done.get(bar, 0)
-                if op == "wait":
-                    assert c < idx + 2, f"{r} waits {bar} phase {idx}, {c} phases already done"
-                    if c <= idx:
-                        break
-                else:
-                    assert idx == c, f"{r}'s arrival on {bar} meant for phase {idx} lands in phase {c}"
-                    pend[bar] = pend.get(bar, 0) + 1
-                    if pend[bar] == counts[bar[0]]:
-                        done[bar], pend[bar] = c + 1, 0
-                cur[r] = next(roles[r], None)
-                progress = True
+
+    def ready(r):
+        op = cur[r]
+        if op is None:
+            return False
+        if op[0] == "wait":
+            assert done.get(op[1], 0) < op[2] + 2, f"{r} waits {op[1]} phase {op[2]}, {done.get(op[1], 0)} done"
+            return done.get(op[1], 0) > op[2]
+        return True
+
+    def execute(r):
+        op, bar, idx = cur[r][:3]
+        if op == "require":
+            missing = [ev for ev in bar if ev not in signalled]
+            assert not missing, f"{r} reuses a buffer before {missing} were signalled"
+        elif op == "arrive":
+            c = done.get(bar, 0)
+            assert idx == c, f"{r}'s arrival on {bar} meant for phase {idx} lands in phase {c}"
+            if len(cur[r]) > 3:
+                pend_ev.setdefault(bar, []).extend(cur[r][3])
+            pend[bar] = pend.get(bar, 0) + 1
+            if pend[bar] == counts[bar[0]]:
+                done[bar], pend[bar] = c + 1, 0
+                signalled.update(pend_ev.pop(bar, []))
+        cur[r] = next(roles[r], None)
+
+    if rng is None:
+        progress = True
+        while progress:
+            progress = False
+            for r in names:
+                while ready(r):
+                    execute(r)
+                    progress = True
+    else:
+        while True:
+            able = [r for r in names if ready(r)]
+            if not able:
+                break
+            execute(rng.choice(able))
     stuck = {r: v for r, v in cur.items() if v is not None}
     assert not stuck, f"deadlock: {stuck}"
 
 
 ORDERS = {
-    "producers first": lambda rs: ["K", "V", "MMA"] + [r for r in rs if r.startswith("S")],
+    "producers first": lambda rs: ["K", "V"] + [r for r in rs if r.startswith("M")] + [r for r in rs if r.startswith("S")],
     "K first, V last": lambda rs: ["K"] + [r for r in rs if r not in ("K", "V")] + ["V"],
-    "softmax first": lambda rs: [r for r in rs if r.startswith("S")] + ["MMA", "K", "V"],
+    "softmax first": lambda rs: [r for r in rs if r.startswith("S")] + [r for r in rs if r.startswith("M")] + ["K", "V"],
     "reversed": lambda rs: list(reversed(rs)),
 }
 
@@ -167,3 +216,19 @@ def test_random_unit_mixes():
     for _ in range(1500):
         units = [rng.randint(1, 6) for _ in range(rng.randint(1, 7))]
         run(units, rng.choice((1, 2)), ORDERS[rng.choice(list(ORDERS))])
+
+
+@pytest.mark.parametrize("window", [0, 512, 128])
+def test_random_schedules_chunked_prefill(window):
+    rng = random.Random(11 + window)
+    for cta in (0, 100, 147):
+        units = chunked_prefill_units(cta, window=window)
+        for _ in range(40):
+            run(units, 2, rng=rng)
+
+
+def test_random_schedules_random_units():
+    rng = random.Random(5)
+    for _ in range(400):
+        units = [rng.randint(1, 5) for _ in range(rng.randint(1, 5))]
+        run(units, rng.choice((1, 2)), rng=rng)
