@@ -57,15 +57,15 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by workload, with the
 # hash of the kernel sources it was taken on; reported only while they match.
 TRAFFIC = {
-    # decode_mma_kernel: 1205.20 MB per launch at batch 32 (the capture-size case, same partitions
-    # as the bench launch), 1.0039 x its algorithmic bytes; scaled to batch 64 (2346.50 MB)
-    "llama2_7b_mha_decode": {"bytes": 2355600000, "kernel_sha": "96e1f88fb35756e9"},
-    # decode_mma_kernel (GQA, 8 query heads per KV head): 694.20 MB per launch at batch 64 (same
-    # partitions as the bench launch), 1.0079 x its algorithmic bytes; scaled to batch 128 (1396.15 MB)
-    "llama2_70b_gqa_decode": {"bytes": 1407200000, "kernel_sha": "96e1f88fb35756e9"},
-    # decode_mma_kernel (int8 codes + fp16 scales): the bench launch itself, 1098.35 MB (1.0071 x its
+    # decode_mma_kernel: 1204.69 MB per launch at batch 32 (the capture-size case, same partitions
+    # as the bench launch), 1.0034 x its algorithmic bytes; scaled to batch 64 (2346.50 MB)
+    "llama2_7b_mha_decode": {"bytes": 2354590000, "kernel_sha": "d9cce3085c6f990f"},
+    # decode_mma_kernel (GQA, 8 query heads per KV head): 693.36 MB per launch at batch 64 (same
+    # partitions as the bench launch), 1.0067 x its algorithmic bytes; scaled to batch 128 (1396.15 MB)
+    "llama2_70b_gqa_decode": {"bytes": 1405480000, "kernel_sha": "d9cce3085c6f990f"},
+    # decode_mma_kernel (int8 codes + fp16 scales): the bench launch itself, 1098.45 MB (1.0072 x its
     # algorithmic bytes, split partials included)
-    "long_ctx_split_kv_int8": {"bytes": 1098350000, "kernel_sha": "96e1f88fb35756e9"},
+    "long_ctx_split_kv_int8": {"bytes": 1098450000, "kernel_sha": "d9cce3085c6f990f"},
     # prefill_tc_kernel: 54.76 MB read + 3.63 MB written per launch, full workload, cold L2
     "chunked_prefill_shared_prefix": {"bytes": 58394112, "kernel_sha": "19f948ac33e1e7cf"},
     # kv_scatter_kernel: 1120.62 MB per launch at a source batch of 16 (35 476 rows; ~43 MB of the

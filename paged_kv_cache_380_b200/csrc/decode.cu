@@ -55,18 +55,14 @@ constexpr unsigned kFull = 0xffffffffu;
 __device__ __forceinline__ uint32_t s8pair_biased(uint32_t w_biased, uint32_t sel_a, uint32_t sel_b) {
     return __byte_perm(w_biased, 0x64646464u, sel_a | 0x40u | (sel_b << 8) | 0x4000u);
 }
-// ... and the code itself: 1152 subtracted from both halves (exact in fp16).  Keys
-// use this form: a key bias would add 1152 sum(q) to every score, and removing it
-// after the fp32 accumulation costs precision when |q| is large.
-__device__ __forceinline__ uint32_t s8pair(uint32_t w_biased, uint32_t sel_a, uint32_t sel_b) {
-    const uint32_t h = s8pair_biased(w_biased, sel_a, sel_b);
-    __half2 x = *reinterpret_cast<const __half2*>(&h);
-    x = __hsub2(x, __half2half2(__ushort_as_half(0x6480)));   // 0x6480 = 1152.0
-    return *reinterpret_cast<uint32_t*>(&x);
-}
-// Values stay biased: sum_t p_t (v_t + 1152) = sum_t p_t v_t + 1152 sum_t p_t, and
-// sum_t p_t comes from one more MMA per chunk against a matrix of ones (the same fp16
-// P operand, p <= 1), accumulated and rescaled with O and subtracted at the end.
+// Both operands stay biased, which saves a subtraction per code pair:
+//  * keys: sum_d q_d (k_d + 1152) = sum_d q_d k_d + 1152 sum_d q_d, so each score
+//    accumulator starts from -1152 sum_d q_d (of the fp16 q the MMAs see) and the bias
+//    cancels inside the fp32 accumulation (measured: the same error against the oracle
+//    as subtracting 1152 from every code, also for all-positive queries);
+//  * values: sum_t p_t (v_t + 1152) = sum_t p_t v_t + 1152 sum_t p_t, and sum_t p_t
+//    comes from one more MMA per chunk against a matrix of ones (the same fp16 P
+//    operand, p <= 1), accumulated and rescaled with O and subtracted at the end.
 constexpr float kCodeBias = 1152.f;
 constexpr uint32_t kOnePair = 0x3C003C00u;    // fp16x2 (1, 1)
 
@@ -103,7 +99,8 @@ template <typename QT, typename KVT, int HD, int NT, int WARPS, int STAGES>
 __global__ void __launch_bounds__(WARPS * 32)
 decode_mma_kernel(const DecodeParams p) {
     using Cfg = DecodeCfg<QT, KVT, HD, NT, WARPS, STAGES>;
-    // INT8 pages run the MMAs in fp16 (codes widen to fp16 in two instructions per pair)
+    // INT8 pages run the MMAs in fp16 (codes widen to fp16, offset by 1152, in one byte
+    // permute per pair after one XOR per four codes)
     using MT = typename std::conditional<Cfg::kInt8, __half, QT>::type;
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -183,6 +180,28 @@ decode_mma_kernel(const DecodeParams p) {
             const float inv = 1.f / f;                                    // exact: a power of two
             qinv[nt][0] = __shfl_sync(kFull, inv, (2 * c) * 4);
             qinv[nt][1] = __shfl_sync(kFull, inv, (2 * c + 1) * 4);
+        }
+    }
+    // INT8 pages: keys widen to 1152 + code, so every score of head n carries 1152 sum_d q_nd;
+    // the accumulators start from minus that (of the fp16 q the MMAs see).
+    float kbias[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) kbias[nt][0] = kbias[nt][1] = 0.f;
+    if constexpr (Cfg::kInt8) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            float sq = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < Cfg::kDT; ++kk)
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const float2 v = unpack2<__half>(qf[nt][kk][i]);
+                    sq += v.x + v.y;
+                }
+            sq += __shfl_xor_sync(kFull, sq, 1);
+            sq += __shfl_xor_sync(kFull, sq, 2);
+            kbias[nt][0] = -kCodeBias * __shfl_sync(kFull, sq, (2 * c) * 4);
+            kbias[nt][1] = -kCodeBias * __shfl_sync(kFull, sq, (2 * c + 1) * 4);
         }
     }
 
@@ -276,7 +295,10 @@ decode_mma_kernel(const DecodeParams p) {
         // ---- S^T = K . Q^T  (16 tokens x 8 heads per n-tile) ----
         float s[NT][4];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+        for (int nt = 0; nt < NT; ++nt) {
+            s[nt][0] = s[nt][2] = kbias[nt][0];
+            s[nt][1] = s[nt][3] = kbias[nt][1];
+        }
         {
             const int r = lane & 15;
             if constexpr (!Cfg::kInt8) {
@@ -298,10 +320,10 @@ decode_mma_kernel(const DecodeParams p) {
                     // w0: rows 0-7 unit U, w1: rows 8-15 unit U, w2/w3: unit U+1
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
-                        mma16816<MT>(s[nt], s8pair(w0, 0, 1), s8pair(w1, 0, 1), s8pair(w0, 2, 3),
-                                     s8pair(w1, 2, 3), qf[nt][U][0], qf[nt][U][1]);
-                        mma16816<MT>(s[nt], s8pair(w2, 0, 1), s8pair(w3, 0, 1), s8pair(w2, 2, 3),
-                                     s8pair(w3, 2, 3), qf[nt][U + 1][0], qf[nt][U + 1][1]);
+                        mma16816<MT>(s[nt], s8pair_biased(w0, 0, 1), s8pair_biased(w1, 0, 1), s8pair_biased(w0, 2, 3),
+                                     s8pair_biased(w1, 2, 3), qf[nt][U][0], qf[nt][U][1]);
+                        mma16816<MT>(s[nt], s8pair_biased(w2, 0, 1), s8pair_biased(w3, 0, 1), s8pair_biased(w2, 2, 3),
+                                     s8pair_biased(w3, 2, 3), qf[nt][U + 1][0], qf[nt][U + 1][1]);
                     }
                 }
             }
