@@ -67,6 +67,48 @@ def test_split_planner_on_the_workloads(lib):
     assert ops.decode_plan(2, 4, 2, 64, 16, 7, torch.float32) == (1, 112)
 
 
+def test_split_planner_properties(lib):
+    """Random shapes: the partitions cover the longest context with none left empty, hold whole
+    pages, never go below 256 tokens or above 2048 (or one page) unless the caller asks for a
+    split count, shorten only while the grid is small (under 12 CTAs per SM above 512 tokens,
+    under 3 above 256; the host reports 148 SMs when no GPU is visible), grow with the number of
+    (sequence, KV head) units, and the workspace is sized for exactly that plan."""
+    import random
+    rng = random.Random(3)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 148
+    dtypes = (torch.bfloat16, torch.float16, torch.int8, torch.float32)
+    for _ in range(3000):
+        B, Hkv = rng.randint(1, 300), rng.choice((1, 2, 4, 8, 16, 32, 64))
+        Hq, D = Hkv * rng.choice((1, 2, 4, 8)), rng.choice((64, 128))
+        ps, mp = rng.choice((16, 32, 64, 128, 256)), rng.randint(1, 1500)
+        dt = rng.choice(dtypes)
+        ns = 0 if rng.random() < 0.7 else rng.randint(1, 80)
+        tokens = mp * ps
+        s, t = ops.decode_plan(B, Hq, Hkv, D, ps, mp, dt, num_splits=ns)
+        assert s >= 1 and t > 0 and t % 16 == 0
+        assert s * t >= tokens and (s - 1) * t < tokens, (B, Hkv, ps, mp, dt, ns, s, t)
+        if dt == torch.float32:
+            assert s == 1
+        else:
+            assert t % ps == 0
+            if ns > 0:
+                assert s <= ns
+            else:
+                assert 256 <= t <= max(2048, ps)
+                if ps == 16:                       # no rounding to whole pages: the fill rule exactly
+                    ctas = B * Hkv * s
+                    assert t == 256 or ctas >= 3 * sms
+                    assert t <= 512 or ctas >= 12 * sms
+                    if t < 2048:                   # halved: the longer partition left the grid small
+                        c2 = B * Hkv * -(-tokens // (2 * t))
+                        assert c2 < 12 * sms if 2 * t > 512 else c2 < 3 * sms
+                    s2, t2 = ops.decode_plan(B + 1, Hq, Hkv, D, ps, mp, dt)
+                    assert t2 >= t
+        rows = B * Hq * s
+        want = 0 if s <= 1 else (rows * D * 4 + 255) // 256 * 256 + rows * 4
+        assert ops.decode_workspace_size(B, Hq, Hkv, D, ps, mp, dt, num_splits=ns) == want
+
+
 def test_workspace_size_matches_plan(lib):
     s, _ = ops.decode_plan(4, 32, 8, 128, 256, 512, torch.bfloat16)
     rows = 4 * 32 * s
