@@ -121,3 +121,16 @@ def test_cpu_baseline_reports_all_cores_and_one_thread():
     got = bench.cpu_baseline(step, budget_s=0.2)
     assert got["unit"] == "TFLOP/s" and got["single_thread"]["cores"] == 1
     assert oracle.max_threads() == threads
+
+
+def test_traffic_figures_belong_to_the_current_kernels():
+    """Every DRAM-traffic figure bench.py can attach was captured on the kernel sources now in
+    the tree (bench.py drops a figure whose source hash differs; this keeps none stale)."""
+    import bench
+    kind_of = {"llama2_7b_mha_decode": "decode", "llama2_70b_gqa_decode": "decode",
+               "long_ctx_split_kv_int8": "decode", "chunked_prefill_shared_prefix": "prefill",
+               "kv_cache_write_full": "scatter"}
+    assert set(bench.TRAFFIC) == set(kind_of)
+    for workload, tr in bench.TRAFFIC.items():
+        assert tr["bytes"] > 0
+        assert tr["kernel_sha"] == bench.kernel_sha(kind_of[workload]), workload
